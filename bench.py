@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the paged MLA decode hot path on B200.
+
+One step = one pass of the whole path over one batch: page table (build_block_table),
+split plan (get_mla_metadata) and attention with its split merge (mla_decode_paged),
+on inputs resident in HBM.  Default workload: the DeepSeek-V3-shaped decode (bs 64,
+128 heads, q_len 1, L ~ U[1024, 4096], bf16 latent KV 576 wide, 64-token pages in a
+shuffled pool 1.25x the need).  L2 is flushed (a 512 MB write) between timed steps,
+outside the step's CUDA events.
+
+Reported (one JSON line on rank 0):
+  value        aggregate KV GB/s over all ranks: algorithmic KV bytes (each request's
+               KV read once) per step x ranks / max-over-ranks step time;
+  roofline     the attention call (decode kernel + merge) against the measured HBM peak:
+               algorithmic (KV + Q) bytes / its CUDA-event time;
+  e2e          the same metric through the public API with the step's inputs (q,
+               seq_lens, req_pool_indices) copied from pinned host memory and the
+               outputs (o, lse) copied back inside the timed region;
+  cpu_baseline the CPU fp64 oracle on a bounded sample of the same workload (rank 0, N=1).
+Multi-GPU: independent replicas (the path has no exchange step); NCCL is used only for
+the barrier and the max-over-ranks reduction of the timings.
+
+--impl reference times the CPU oracle (the reference arm) on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged MLA decode: KV GB/s, TFLOP/s and % roofline; µs per call"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 4  # page table, planner, attention, split merge
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--flush-mb", type=int, default=512)
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(config: int, rank: int) -> int:
+    """Each replica owns its own pool and batch: distinct seeds per rank."""
+    return 1000 + config + 100 * rank
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(wl):
+    """KV bytes (each request's KV once), Q bytes and FLOPs of one attention call."""
+    elem = 1 if wl.is_fp8 else 2
+    L = [int(x) for x in wl.cache_seqlens.tolist()]
+    kv = sum(L) * 576 * elem
+    qb = wl.bs * wl.q_len * wl.h * 576 * 2
+    flops = 0
+    for Lb in L:
+        for i in range(wl.q_len):
+            allowed = max(0, min(Lb, Lb - wl.q_len + i + 1)) if wl.causal else Lb
+            flops += 2 * wl.h * allowed * (576 + 512)
+    return kv, qb, flops
+
+
+def workload_config(cfg_index, wl, world, flush_mb):
+    from paged_kv_mla_create_b200.workloads import CONFIGS
+    c = CONFIGS[cfg_index]
+    return {"workload": c["name"], "batch": wl.bs, "heads": wl.h, "q_len": wl.q_len,
+            "kv_dtype": "fp8_e4m3" if wl.is_fp8 else "bf16", "page": 64,
+            "head_dim": 576, "head_dim_v": 512,
+            "l2": f"flushed between timed steps ({flush_mb} MB write, outside the step events)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [l.strip().split(",") for l in self.out.read().splitlines() if l.strip()]
+        os.unlink(self.out.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 10:
+                continue
+            try:
+                sm.append(float(r[2]))
+                smax.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id_for(device) -> str:
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(device).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return str(device.index or 0)
+
+
+def _oracle_rows(wl, rows):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.mla_decode_rows(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
+                           wl.cache_seqlens, rows, wl.softmax_scale, wl.causal,
+                           kv_is_fp8=wl.is_fp8,
+                           descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
+                           descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+    return time.perf_counter() - t0
+
+
+def _row_sample(wl, n):
+    """n query rows spread evenly over all requests and heads."""
+    import numpy as np
+    total = wl.bs * wl.q_len * wl.h
+    n = int(max(1, min(total, n)))
+    return np.unique(np.linspace(0, total - 1, n).round().astype(np.int64))
+
+
+def _calibrate(wl):
+    """Rows per second of the oracle on this host (one row per request)."""
+    rows = _row_sample(wl, wl.bs)
+    return len(rows) / max(_oracle_rows(wl, rows), 1e-6)
+
+
+def cpu_baseline(wl, seconds):
+    """The oracle as it stands on the host cores, on a bounded sample of rows spread over
+    all requests and heads, scaled to KV GB/s by the fraction of rows processed."""
+    import oracle
+    kv_bytes, _, _ = algorithmic(wl)
+    total = wl.bs * wl.q_len * wl.h
+    rows = _row_sample(wl, _calibrate(wl) * seconds)
+    dt = _oracle_rows(wl, rows)
+    frac = len(rows) / total
+    return {"value": kv_bytes * frac / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {total} query rows spread over all {wl.bs} requests, "
+                      f"{dt:.1f} s; KV bytes scaled by the row fraction {frac:.4f}"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, K timed steps of a bounded row sample each,
+    sized so that warm-up plus timed steps take about two minutes of host time."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from paged_kv_mla_create_b200 import workloads as W
+    wl = W.make_workload(args.config, seed=replica_seed(args.config, 0))
+    kv_bytes, _, _ = algorithmic(wl)
+    total = wl.bs * wl.q_len * wl.h
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    rows = _row_sample(wl, _calibrate(wl) * per_step)
+    for _ in range(args.warmup):
+        _oracle_rows(wl, rows)
+    times = [_oracle_rows(wl, rows) for _ in range(args.steps)]
+    sec = statistics.median(times)
+    frac = len(rows) / total
+    value = kv_bytes * frac / sec / 1e9
+    sample = (f"{len(rows)} of {total} query rows per step spread over all {wl.bs} requests; "
+              f"KV bytes scaled by the row fraction {frac:.5f}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args.config, wl, 1, 0),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_mla_create_b200 as mla
+    from paged_kv_mla_create_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    mla.library()
+
+    host = W.make_workload(args.config, seed=replica_seed(args.config, rank))
+    wl = host.to(dev)
+    kv_bytes, q_bytes, flops = algorithmic(host)
+    bs, q_len, h = host.bs, host.q_len, host.h
+    parts = mla.num_sm_parts(q_len * h, 1, mla.sm_count(dev))
+    bt = torch.empty((bs, host.max_pages), dtype=torch.int32, device=dev)
+    md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
+    ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
+    o = torch.empty((bs, q_len, h, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((bs, q_len, h), dtype=torch.float32, device=dev)
+    ws = torch.empty((mla.workspace_bytes(bs, q_len, h, parts),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((args.flush_mb << 20,), dtype=torch.uint8, device=dev)
+
+    def metadata(w):
+        mla.build_block_table(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
+                              seq_len_add=host.num_draft_tokens, out=bt)
+        mla.get_mla_metadata(w.cache_seqlens, q_len * h, 1, host.is_fp8, num_parts=parts,
+                             out=(md, ns))
+
+    def attention(w):
+        mla.mla_decode_paged(w.q, w.kv_cache, bt, w.cache_seqlens, 512, md, ns,
+                             host.softmax_scale, host.causal, w.descale_q, w.descale_k,
+                             out=o, lse=lse, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        metadata(wl)
+        attention(wl)
+    torch.cuda.synchronize(dev)
+    if mla.read_device_error(dev) != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(gpu_id_for(dev))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record(stream)
+        metadata(wl)
+        ev[k][1].record(stream)
+        attention(wl)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / K
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    meta_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+
+    # end to end through the public API, host buffers in and out
+    pin_q = host.q.pin_memory()
+    pin_sl = host.seq_lens.pin_memory()
+    pin_cl = host.cache_seqlens.pin_memory()
+    pin_rpi = host.req_pool_indices.pin_memory()
+    out_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    out_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    dq = torch.empty_like(wl.q)
+    dsl = torch.empty_like(wl.seq_lens)
+    dcl = torch.empty_like(wl.cache_seqlens)
+    drpi = torch.empty_like(wl.req_pool_indices)
+    import dataclasses
+    we = dataclasses.replace(wl, q=dq, seq_lens=dsl, cache_seqlens=dcl, req_pool_indices=drpi)
+    h2d = sum(t.numel() * t.element_size() for t in (pin_q, pin_sl, pin_cl, pin_rpi))
+    d2h = out_o.numel() * out_o.element_size() + out_lse.numel() * out_lse.element_size()
+    KE = max(1, min(args.e2e_steps, K))
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(KE)]
+    torch.cuda.synchronize(dev)
+    for k in range(KE):
+        flush.fill_(k & 0xFF)
+        ee[k][0].record(stream)
+        dq.copy_(pin_q, non_blocking=True)
+        dsl.copy_(pin_sl, non_blocking=True)
+        dcl.copy_(pin_cl, non_blocking=True)
+        drpi.copy_(pin_rpi, non_blocking=True)
+        metadata(we)
+        attention(we)
+        out_o.copy_(o, non_blocking=True)
+        out_lse.copy_(lse, non_blocking=True)
+        ee[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in ee) / KE
+    err = mla.read_device_error(dev)
+
+    t = torch.tensor([step_ms, attn_ms, meta_ms, e2e_ms, float(err)], dtype=torch.float64,
+                     device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, attn_ms, meta_ms, e2e_ms, err = t.tolist()
+    if err:
+        raise RuntimeError(f"device error word {int(err)} after the timed run")
+
+    peaks, peak_src = load_peaks()
+    t_hbm = (kv_bytes + q_bytes) / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    attn_s = attn_ms * 1e-3
+    achieved_gbs = (kv_bytes + q_bytes) / attn_s / 1e9
+    achieved_tf = flops / attn_s / 1e12
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"]}
+    roof.update({"traffic": None, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
+                 if peak_src == "measured" else "fallback",
+                 "kernel": "mla_decode_paged call (decode kernel + split merge)",
+                 "roofline_time_us": max(t_hbm, t_tc) * 1e6,
+                 "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s})
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+    value = world * kv_bytes / (step_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(args.config, host, world, args.flush_mb),
+        "us_per_call": attn_ms * 1e3, "metadata_us": meta_ms * 1e3,
+        "kv_gbs_per_call": kv_bytes / attn_s / 1e9, "tflops": achieved_tf,
+        "tensor_frac": achieved_tf / peaks["bf16_tflops"],
+        "roofline": roof,
+        "e2e": {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(host, args.cpu_seconds)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_b200(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,219 @@
+/*
+ * mla_b200.h — C ABI of the B200 (sm_100a) paged MLA decode library.
+ *
+ * Three operations, in the order a decode step calls them, each in the role the
+ * SGLang FlashMLA attention backend page (flashmla_backend.py) gives it:
+ *
+ *   mla_build_block_table  the per-request page table of
+ *                          FlashMLABackend.init_forward_metadata (decode and
+ *                          target-verify branches, create_flashmla_kv_indices_triton);
+ *   mla_get_mla_metadata   the split-KV scheduler of get_mla_metadata
+ *                          (tile_scheduler_metadata [num_sm_parts, 8], num_splits [bs+1]);
+ *   mla_decode_paged       the attention of flash_mla_with_kvcache as called by
+ *                          forward_decode / forward_extend (target-verify), with the
+ *                          log-sum-exp merge of KV splits.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller (for example a
+ *     torch tensor's data_ptr()), unless its comment says "host".  The library keeps
+ *     no state between calls and allocates no device memory: scratch space is the
+ *     caller's `workspace`.  Every call is asynchronous on `stream` (NULL = the legacy
+ *     default stream), makes no host synchronisation and no allocation, and may
+ *     therefore be captured in a CUDA graph.
+ *   - Arguments are validated on the host before any launch; a violation returns
+ *     MLA_ERR_INVALID_ARG (or MLA_ERR_UNSUPPORTED for a valid but unimplemented
+ *     combination) and launches nothing.  A CUDA launch error returns MLA_ERR_CUDA.
+ *   - Facts only the device can see (a page id outside the pool, a request-pool row
+ *     outside req_to_token, a length beyond the page table, a malformed scheduler row,
+ *     a pipeline wait that timed out) never fault: the kernel skips or clamps the
+ *     access and ORs a bit into a sticky device error word, which
+ *     mla_read_device_error returns and clears.
+ *   - bs == 0 (the idle batch) returns MLA_OK and launches nothing.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,   /* an argument is out of its documented range     */
+    MLA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, head dims)    */
+    MLA_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed             */
+    MLA_ERR_DEVICE_CHECK = 4,  /* mla_read_device_error found a device-side error */
+    MLA_ERR_WORKSPACE = 5      /* workspace missing or smaller than required      */
+} mla_status_t;
+
+/* Element / index types. */
+enum {
+    MLA_DTYPE_BF16 = 0,
+    MLA_DTYPE_FP8_E4M3 = 1,    /* OCP e4m3 "fn": no infinities, S.1111.111 = NaN */
+    MLA_DTYPE_INT32 = 2,
+    MLA_DTYPE_INT64 = 3
+};
+
+/* Bits of the sticky device error word (mla_read_device_error). */
+enum {
+    MLA_DEVERR_PAGE_OUT_OF_RANGE = 1,  /* block-table page id not in [0, num_pages): tile read as zeros */
+    MLA_DEVERR_ROW_OUT_OF_RANGE = 2,   /* req_pool_indices[b] not a row of req_to_token: row skipped   */
+    MLA_DEVERR_LEN_OUT_OF_RANGE = 4,   /* a length exceeds the table / req_to_token width: clamped     */
+    MLA_DEVERR_BAD_METADATA = 8,       /* a scheduler row is not a valid cursor range: part skipped    */
+    MLA_DEVERR_WAIT_TIMEOUT = 16       /* a pipeline wait exceeded its bound: the CTA gave up          */
+};
+
+typedef struct CUstream_st* mla_stream_t;  /* identical to cudaStream_t */
+
+/* Human-readable name of a status code (static storage, never NULL). */
+MLA_API const char* mla_status_string(mla_status_t status);
+
+/* Version of this ABI; bumped whenever a signature or layout below changes. */
+MLA_API int32_t mla_abi_version(void);
+
+/*
+ * Page table (flashmla_backend.py, init_forward_metadata: block_kv_indices of shape
+ * [bs, cdiv(max L, 64)], int32, pre-filled with -1, filled from req_to_token,
+ * req_pool_indices and seq_lens; the target-verify branch first adds
+ * num_draft_tokens to every length).
+ *
+ * For request b with L_b = seq_lens[b] + seq_len_add and every page p < cdiv(L_b, page_size):
+ *     block_table[b * block_table_stride + p] =
+ *         req_to_token[req_pool_indices[b] * req_to_token_stride + p * page_size] / page_size
+ * (the pool viewed [-1, page_size, 1, 576] puts slots page_size*P .. page_size*P+page_size-1
+ * in page P, so slots must be page-aligned and in order inside a page).
+ * Entries p in [cdiv(L_b, page_size), max_pages) are written with -1 when fill_tail != 0
+ * and left untouched otherwise (the caller's pre-fill, as in the graph-capture path).
+ *
+ *   req_to_token         int32 [req_to_token_rows, req_to_token_stride] (row-major)
+ *   req_pool_indices     [bs], int32 or int64 (rpi_dtype)
+ *   seq_lens             [bs], int32 or int64 (seq_lens_dtype)
+ *   block_table          int32 [bs, block_table_stride], written for p < max_pages
+ *   page_size            must be 64
+ * Device checks: a row index outside [0, req_to_token_rows) leaves the row at -1 and
+ * sets MLA_DEVERR_ROW_OUT_OF_RANGE; L_b beyond max_pages pages or beyond
+ * req_to_token_stride positions is clamped and sets MLA_DEVERR_LEN_OUT_OF_RANGE.
+ */
+MLA_API mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t req_to_token_rows,
+                                   int64_t req_to_token_stride, const void* req_pool_indices,
+                                   int32_t rpi_dtype, const void* seq_lens, int32_t seq_lens_dtype,
+                                   int32_t seq_len_add, int32_t bs, int32_t* block_table,
+                                   int64_t block_table_stride, int32_t max_pages,
+                                   int32_t page_size, int32_t fill_tail, mla_stream_t stream);
+
+/*
+ * Number of scheduler parts (the first dimension of tile_scheduler_metadata) for
+ * get_mla_metadata(cache_seqlens, num_heads_per_head_k, num_heads_k): every part is
+ * served by a pair of SMs per 128-row query tile, so
+ *     num_sm_parts = max(1, sm_count / (2 * cdiv(num_heads_per_head_k, 128) * num_heads_k)).
+ * num_heads_per_head_k is q_len * h_q (num_draft_tokens * h_q in target-verify, as the
+ * backend passes it); num_heads_k is 1 for MLA.  Returns -1 on a non-positive argument.
+ * Pure host function.
+ */
+MLA_API int32_t mla_num_sm_parts(int32_t sm_count, int32_t num_heads_per_head_k, int32_t num_heads_k);
+
+/*
+ * Split-KV scheduler (flashmla_backend.py, get_mla_metadata: tile_scheduler_metadata
+ * int32 [num_sm_parts, 8], num_sm_parts <= the SM count, and num_splits int32 [bs+1]).
+ * The pages fix only these shapes; the contents are defined here:
+ *   blocks_b = cdiv(cache_seqlens[b], 64); each piece of a request costs its blocks plus
+ *   a fixed overhead of 5 blocks; total = sum_b (blocks_b + 5); every part has the budget
+ *   cdiv(total, num_sm_parts) + 5 and is filled greedily in request order: a request that
+ *   fits in what is left is taken whole, otherwise the part takes (budget - 5) blocks of it
+ *   when that is positive, and ends.
+ *   Row i = [begin_req, begin_block, end_req, end_block, begin_split, 0, 0, 0], where
+ *   (end_req, end_block) is the exclusive cursor after the part and begin_split the index
+ *   of the part's first piece within its request; num_splits[0] = 0 and
+ *   num_splits[b+1] - num_splits[b] = number of pieces of request b.
+ * Every block of every request is covered exactly once within num_sm_parts parts, and
+ * num_splits[bs] <= bs + num_sm_parts - 1.
+ *   cache_seqlens          int32 [bs] (negative lengths count as 0)
+ *   num_sm_parts           from mla_num_sm_parts (>= 1)
+ *   is_fp8_kvcache         accepted; it does not change the plan
+ *   tile_scheduler_metadata int32 [num_sm_parts, 8] (written)
+ *   num_splits             int32 [bs + 1] (written)
+ * One single-CTA launch; bs must be <= 1,048,576.
+ */
+MLA_API mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
+                                  int32_t num_sm_parts, int32_t is_fp8_kvcache,
+                                  int32_t* tile_scheduler_metadata, int32_t* num_splits,
+                                  mla_stream_t stream);
+
+/*
+ * Bytes of workspace mla_decode_paged needs: partial outputs fp32
+ * [(bs + num_sm_parts) * q_len * h_q, 512] and their log-sum-exps, 256-byte aligned.
+ * Pure host function; returns 0 on a non-positive argument.
+ */
+MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q, int32_t num_sm_parts);
+
+/*
+ * Paged MLA attention (flashmla_backend.py, forward_decode / forward_extend:
+ * flash_mla_with_kvcache(q, k_cache.view(-1, 64, 1, 576), block_table, cache_seqlens,
+ * head_dim_v = kv_lora_rank, tile_scheduler_metadata, num_splits, softmax_scale,
+ * causal, descale_q, descale_k)).
+ *
+ * For every request b, query position i < q_len and head h (row r = i * h_q + h):
+ *   L = cache_seqlens[b]; keys j < lim with lim = L - q_len + i + 1 when causal
+ *   (the draft tokens are the last q_len positions of the cache) and lim = L otherwise;
+ *   k_j = KV row of position j (through block_table, page j / 64, row j % 64) * descale_k;
+ *   v_j = k_j[0:512];  s_j = softmax_scale * descale_q * <q[b,i,h,:], k_j>;
+ *   lse = ln sum_j exp(s_j);  o = sum_j exp(s_j - lse) v_j.
+ *   A row with no allowed key gets o = 0 and lse = -inf.
+ *
+ *   q                 bf16 [bs, q_len, h_q, head_dim], contiguous
+ *   q_dtype           MLA_DTYPE_BF16
+ *   head_dim          576 (kv_lora_rank 512 + qk_rope_head_dim 64); head_dim_v 512
+ *   k_cache           [num_pages, page_size, head_dim] bf16 or e4m3 (kv_dtype), contiguous;
+ *                     every value must be finite (tail rows of a page are read and masked)
+ *   page_size         64
+ *   block_table       int32 [bs, block_table_stride]; entries p < cdiv(L, 64) are read
+ *   max_pages         usable columns of block_table (L must be <= 64 * max_pages)
+ *   cache_seqlens     int32 [bs]
+ *   tile_scheduler_metadata, num_splits  from mla_get_mla_metadata for the same
+ *                     cache_seqlens and num_sm_parts, with num_sm_parts from
+ *                     mla_num_sm_parts(sm_count, q_len * h_q, 1)
+ *   softmax_scale     host float (1/sqrt(192) for DeepSeek-V3)
+ *   causal            0 or 1
+ *   descale_q, descale_k  device fp32 [1]; NULL means 1.0.  descale_k scales the fp8
+ *                     cache values; descale_q scales q.
+ *   out               bf16 [bs, q_len, h_q, 512] (written)
+ *   lse               fp32 [bs, q_len, h_q] natural-log log-sum-exp (written)
+ *   workspace         at least mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts)
+ *                     bytes, 256-byte aligned; its contents need no initialisation
+ * Calls on the same workspace that overlap on the GPU race; use one workspace per stream.
+ * The first call on a device also sets the kernel's shared-memory limit (a host-side
+ * attribute; no allocation).
+ */
+MLA_API mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_t q_len,
+                              int32_t h_q, int32_t head_dim, int32_t head_dim_v,
+                              const void* k_cache, int32_t kv_dtype, int64_t num_pages,
+                              int32_t page_size, const int32_t* block_table,
+                              int64_t block_table_stride, int32_t max_pages,
+                              const int32_t* cache_seqlens, const int32_t* tile_scheduler_metadata,
+                              int32_t num_sm_parts, const int32_t* num_splits, float softmax_scale,
+                              int32_t causal, const float* descale_q, const float* descale_k,
+                              void* out, float* lse, void* workspace, size_t workspace_bytes,
+                              mla_stream_t stream);
+
+/*
+ * Read and clear the sticky device error word of the current device (a bitwise OR of
+ * MLA_DEVERR_* since the last read).  Synchronises `stream`, so it is not for use inside
+ * graph capture.  *code_out (host) receives the word; returns MLA_ERR_DEVICE_CHECK when it
+ * is non-zero, MLA_OK when it is zero.
+ */
+MLA_API mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

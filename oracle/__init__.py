@@ -68,6 +68,8 @@ def _load():
     lib.oracle_e4m3_to_double.restype = D
     lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_double.restype = D
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = I32
     _lib = lib
     return lib
 
@@ -85,6 +87,11 @@ def _np(x, dtype):
 
 def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().oracle_num_threads())
 
 
 def e4m3_to_double(code: int) -> float:

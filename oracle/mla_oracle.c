@@ -29,6 +29,7 @@
  *                             ragged and a paged partial result).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -55,6 +56,9 @@ static double e4m3_bits_to_double(uint8_t bits) {
         v = ldexp((double)(8 + m), e - 10);  /* (1 + m/8) * 2^(e-7) */
     return sign ? -v : v;
 }
+
+/* Threads the OpenMP loops use (the host's cores unless OMP_NUM_THREADS says otherwise). */
+int oracle_num_threads(void) { return omp_get_max_threads(); }
 
 double oracle_e4m3_to_double(uint8_t bits) { return e4m3_bits_to_double(bits); }
 double oracle_bf16_to_double(uint16_t bits) { return bf16_bits_to_double(bits); }

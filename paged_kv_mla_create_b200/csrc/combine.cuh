@@ -1,0 +1,66 @@
+// Log-sum-exp merge of split-KV partial results: the step implied by get_mla_metadata's
+// num_splits in the SGLang FlashMLA backend page (flashmla_backend.py) and written out
+// as merge_state on the FlashInfer backend page (flashinfer_backend.py, forward_extend):
+//     lse = ln sum_i exp(lse_i),   o = sum_i exp(lse_i - lse) * o_i.
+//
+// One warp per (request, query row).  Requests with a single piece were written
+// directly by the attention kernel and are skipped here, so the launch needs no host
+// knowledge of the plan.  A warp reads its pieces' lse values, then streams the
+// pieces' 512 fp32 columns (16 per lane, as 4 float4) and writes bf16.
+#pragma once
+#include "ptx.cuh"
+
+namespace mla {
+
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                      const int32_t* __restrict__ num_splits, int32_t rows,
+                      __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+    const int b = blockIdx.y;
+    const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int s0 = num_splits[b];
+    const int n = num_splits[b + 1] - s0;
+    if (n <= 1) return;
+    float m = -INFINITY;
+    for (int i = lane; i < n; i += 32) m = fmaxf(m, part_lse[(int64_t)(s0 + i) * rows + row]);
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const int64_t out_row = (int64_t)b * rows + row;
+    if (m == -INFINITY) {
+        for (int c = lane; c < 64; c += 32)
+            reinterpret_cast<uint4*>(out + out_row * 512)[c] = make_uint4(0, 0, 0, 0);
+        if (lane == 0) lse_out[out_row] = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int i = lane; i < n; i += 32) sum += expf(part_lse[(int64_t)(s0 + i) * rows + row] - m);
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float lse = m + logf(sum);
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (int i = 0; i < n; ++i) {
+        const float li = part_lse[(int64_t)(s0 + i) * rows + row];
+        const float w = expf(li - lse);
+        const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 v = src[lane + 32 * k];
+            acc[4 * k + 0] += w * v.x;
+            acc[4 * k + 1] += w * v.y;
+            acc[4 * k + 2] += w * v.z;
+            acc[4 * k + 3] += w * v.w;
+        }
+    }
+    uint2* dst = reinterpret_cast<uint2*>(out + out_row * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        dst[lane + 32 * k] = make_uint2(pack_bf16x2(acc[4 * k], acc[4 * k + 1]),
+                                        pack_bf16x2(acc[4 * k + 2], acc[4 * k + 3]));
+    if (lane == 0) lse_out[out_row] = lse;
+}
+
+}  // namespace mla

@@ -1,0 +1,245 @@
+// C ABI of the paged MLA decode library (declared in include/mla_b200.h): host-side
+// argument validation, TMA tensor-map encoding and kernel launches.  The kernels live in
+// the headers included below; this file is the library's only translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla_b200.h"
+#include "block_table.cuh"
+#include "combine.cuh"
+#include "decode.cuh"
+#include "planner.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so that the library
+// links against no driver library at build time and loads on hosts without a GPU.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Per-device one-time setting of the decode kernels' shared-memory limit.
+mla_status_t prepare_decode_kernels() {
+    static std::once_flag flags[kMaxDevices];
+    static cudaError_t results[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    std::call_once(flags[dev], [dev] {
+        results[dev] = cudaFuncSetAttribute(mla::decode::mla_decode_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mla::decode::kSmemBytes);
+    });
+    return from_cuda(results[dev]);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+    switch (s) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+        case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK";
+        case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    }
+    return "MLA_ERR_UNKNOWN";
+}
+
+int32_t mla_abi_version(void) { return 1; }
+
+mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t req_to_token_rows,
+                                   int64_t req_to_token_stride, const void* req_pool_indices,
+                                   int32_t rpi_dtype, const void* seq_lens, int32_t seq_lens_dtype,
+                                   int32_t seq_len_add, int32_t bs, int32_t* block_table,
+                                   int64_t block_table_stride, int32_t max_pages,
+                                   int32_t page_size, int32_t fill_tail, mla_stream_t stream) {
+    if (bs < 0 || max_pages < 0 || page_size != 64) return MLA_ERR_INVALID_ARG;
+    if (rpi_dtype != MLA_DTYPE_INT32 && rpi_dtype != MLA_DTYPE_INT64) return MLA_ERR_INVALID_ARG;
+    if (seq_lens_dtype != MLA_DTYPE_INT32 && seq_lens_dtype != MLA_DTYPE_INT64)
+        return MLA_ERR_INVALID_ARG;
+    if (bs == 0 || max_pages == 0) return MLA_OK;
+    if (!req_to_token || !req_pool_indices || !seq_lens || !block_table) return MLA_ERR_INVALID_ARG;
+    if (req_to_token_rows <= 0 || req_to_token_stride <= 0 || block_table_stride < max_pages)
+        return MLA_ERR_INVALID_ARG;
+    if (bs > 65535) return MLA_ERR_UNSUPPORTED;
+    const dim3 grid(bs, (max_pages + 255) / 256);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define MLA_BT_LAUNCH(IT, LT)                                                                     \
+    mla::build_block_table_kernel<IT, LT><<<grid, 256, 0, st>>>(                                 \
+        req_to_token, req_to_token_rows, req_to_token_stride,                                     \
+        static_cast<const IT*>(req_pool_indices), static_cast<const LT*>(seq_lens), seq_len_add, \
+        block_table, block_table_stride, max_pages, fill_tail)
+    if (rpi_dtype == MLA_DTYPE_INT64 && seq_lens_dtype == MLA_DTYPE_INT64) MLA_BT_LAUNCH(int64_t, int64_t);
+    else if (rpi_dtype == MLA_DTYPE_INT64) MLA_BT_LAUNCH(int64_t, int32_t);
+    else if (seq_lens_dtype == MLA_DTYPE_INT64) MLA_BT_LAUNCH(int32_t, int64_t);
+    else MLA_BT_LAUNCH(int32_t, int32_t);
+#undef MLA_BT_LAUNCH
+    return from_cuda(cudaGetLastError());
+}
+
+int32_t mla_num_sm_parts(int32_t sm_count, int32_t num_heads_per_head_k, int32_t num_heads_k) {
+    if (sm_count <= 0 || num_heads_per_head_k <= 0 || num_heads_k <= 0) return -1;
+    const int32_t m_tiles = (num_heads_per_head_k + 127) / 128;
+    const int32_t parts = sm_count / (2 * m_tiles * num_heads_k);
+    return parts < 1 ? 1 : parts;
+}
+
+mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
+                                  int32_t num_sm_parts, int32_t is_fp8_kvcache,
+                                  int32_t* tile_scheduler_metadata, int32_t* num_splits,
+                                  mla_stream_t stream) {
+    (void)is_fp8_kvcache;  // accepted for call compatibility; the plan does not depend on it
+    if (bs < 0 || num_sm_parts < 1 || bs > (1 << 20)) return MLA_ERR_INVALID_ARG;
+    if (!tile_scheduler_metadata || !num_splits || (bs > 0 && !cache_seqlens))
+        return MLA_ERR_INVALID_ARG;
+    if (!is_aligned(tile_scheduler_metadata, 16)) return MLA_ERR_INVALID_ARG;
+    mla::get_mla_metadata_kernel<<<1, mla::kPlannerThreads, 0,
+                                   reinterpret_cast<cudaStream_t>(stream)>>>(
+        cache_seqlens, bs, num_sm_parts, tile_scheduler_metadata, num_splits);
+    return from_cuda(cudaGetLastError());
+}
+
+size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q, int32_t num_sm_parts) {
+    if (bs <= 0 || q_len <= 0 || h_q <= 0 || num_sm_parts <= 0) return 0;
+    const size_t splits = (size_t)bs + (size_t)num_sm_parts;
+    const size_t rows = (size_t)q_len * (size_t)h_q;
+    return align256(splits * rows * 512 * sizeof(float)) + align256(splits * rows * sizeof(float));
+}
+
+mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_t q_len,
+                              int32_t h_q, int32_t head_dim, int32_t head_dim_v,
+                              const void* k_cache, int32_t kv_dtype, int64_t num_pages,
+                              int32_t page_size, const int32_t* block_table,
+                              int64_t block_table_stride, int32_t max_pages,
+                              const int32_t* cache_seqlens, const int32_t* tile_scheduler_metadata,
+                              int32_t num_sm_parts, const int32_t* num_splits, float softmax_scale,
+                              int32_t causal, const float* descale_q, const float* descale_k,
+                              void* out, float* lse, void* workspace, size_t workspace_bytes,
+                              mla_stream_t stream) {
+    if (bs < 0 || q_len <= 0 || h_q <= 0 || num_sm_parts < 1) return MLA_ERR_INVALID_ARG;
+    if (head_dim != 576 || head_dim_v != 512 || page_size != 64) return MLA_ERR_UNSUPPORTED;
+    if (q_dtype != MLA_DTYPE_BF16) return MLA_ERR_UNSUPPORTED;
+    if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+    if (kv_dtype == MLA_DTYPE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+    if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    if (bs == 0) return MLA_OK;
+    if (!q || !k_cache || !block_table || !cache_seqlens || !tile_scheduler_metadata ||
+        !num_splits || !out || !lse)
+        return MLA_ERR_INVALID_ARG;
+    if (num_pages <= 0 || num_pages * 64 >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+    if (max_pages <= 0 || block_table_stride < max_pages) return MLA_ERR_INVALID_ARG;
+    if ((int64_t)q_len * h_q > (int64_t(1) << 24) || bs > 65535) return MLA_ERR_UNSUPPORTED;
+    if (!is_aligned(q, 16) || !is_aligned(k_cache, 16) || !is_aligned(out, 16) ||
+        !is_aligned(tile_scheduler_metadata, 16))
+        return MLA_ERR_INVALID_ARG;
+    const size_t need = mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts);
+    if (!workspace || workspace_bytes < need || !is_aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+
+    mla_status_t st = prepare_decode_kernels();
+    if (st != MLA_OK) return st;
+    EncodeTiledFn encode = encode_tiled();
+    if (!encode) return MLA_ERR_CUDA;
+
+    // KV pool as a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16, 64 x 64 boxes with
+    // 128-byte swizzle; rows past the end read as zeros.
+    CUtensorMap kv_map;
+    std::memset(&kv_map, 0, sizeof kv_map);
+    const cuuint64_t gdim[2] = {576, (cuuint64_t)num_pages * 64};
+    const cuuint64_t gstride[1] = {576 * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache),
+                         gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return MLA_ERR_CUDA;
+
+    const int32_t rows = q_len * h_q;
+    const size_t splits = (size_t)bs + (size_t)num_sm_parts;
+    mla::decode::Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kv_fp8 = nullptr;
+    p.block_table = block_table;
+    p.bt_stride = block_table_stride;
+    p.max_pages = max_pages;
+    p.cache_seqlens = cache_seqlens;
+    p.md = tile_scheduler_metadata;
+    p.num_splits = num_splits;
+    p.bs = bs;
+    p.q_len = q_len;
+    p.h_q = h_q;
+    p.rows = rows;
+    p.num_pages = num_pages;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.descale_q = descale_q;
+    p.descale_k = descale_k;
+    p.causal = causal;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          align256(splits * rows * 512 * sizeof(float)));
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
+    mla::decode::mla_decode_kernel<false><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
+        kv_map, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    const dim3 cgrid((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
+    mla::combine_splits_kernel<<<cgrid, mla::kCombineWarps * 32, 0, s>>>(
+        p.part_o, p.part_lse, num_splits, rows, p.out, lse);
+    return from_cuda(cudaGetLastError());
+}
+
+mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t stream) {
+    if (!code_out) return MLA_ERR_INVALID_ARG;
+    int value = 0;
+    const int zero = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&value, mla::g_device_error, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(mla::g_device_error, &zero, sizeof(int), 0,
+                                    cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    *code_out = value;
+    return value ? MLA_ERR_DEVICE_CHECK : MLA_OK;
+}
+
+}  // extern "C"

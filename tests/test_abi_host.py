@@ -1,0 +1,102 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every symbol the
+header declares, and its host-only logic (part count, workspace size, argument
+validation) behaves as documented.  No call here reaches a CUDA API."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import paged_kv_mla_create_b200 as mla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla_b200.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = mla.library()
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings():
+    lib = mla.library()
+    assert lib.mla_abi_version() == 1
+    for code, name in mla._STATUS.items():
+        assert lib.mla_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("sm,heads,hk", [(148, 128, 1), (148, 512, 1), (148, 16, 1), (148, 129, 1),
+                                         (132, 128, 1), (1, 128, 1), (148, 128, 2), (148, 4096, 1)])
+def test_num_sm_parts_matches_oracle(sm, heads, hk):
+    assert mla.library().mla_num_sm_parts(sm, heads, hk) == oracle.num_sm_parts(sm, heads, hk)
+
+
+def test_num_sm_parts_rejects_bad_arguments():
+    lib = mla.library()
+    assert lib.mla_num_sm_parts(0, 128, 1) == -1
+    assert lib.mla_num_sm_parts(148, 0, 1) == -1
+    assert lib.mla_num_sm_parts(148, 128, 0) == -1
+
+
+def test_workspace_bytes():
+    lib = mla.library()
+    ws = lib.mla_decode_workspace_bytes(64, 1, 128, 74)
+    rows, splits = 128, 64 + 74
+    expect = -(-splits * rows * 512 * 4 // 256) * 256 + -(-splits * rows * 4 // 256) * 256
+    assert ws == expect
+    assert lib.mla_decode_workspace_bytes(0, 1, 128, 74) == 0
+    assert lib.mla_decode_workspace_bytes(1, 1, 128, 0) == 0
+
+
+def _decode(lib, **over):
+    args = dict(q=1 << 20, q_dtype=0, bs=2, q_len=1, h_q=16, head_dim=576, head_dim_v=512,
+                k_cache=1 << 21, kv_dtype=0, num_pages=8, page_size=64, block_table=1 << 22,
+                bt_stride=3, max_pages=3, cache_seqlens=1 << 23, md=1 << 24, parts=74,
+                num_splits=1 << 25, scale=0.07, causal=1, dq=None, dk=None, out=1 << 26,
+                lse=1 << 27, ws=1 << 28, ws_bytes=1 << 30, stream=None)
+    args.update(over)
+    return lib.mla_decode_paged(*args.values())
+
+
+def test_decode_validation_happens_before_any_launch():
+    lib = mla.library()
+    assert _decode(lib, bs=0) == 0                       # idle batch: nothing to do
+    assert _decode(lib, head_dim=512) == 2               # unsupported head dims
+    assert _decode(lib, head_dim_v=576) == 2
+    assert _decode(lib, page_size=32) == 2
+    assert _decode(lib, q_dtype=1) == 2                  # fp8 q: not implemented
+    assert _decode(lib, kv_dtype=7) == 1
+    assert _decode(lib, causal=2) == 1
+    assert _decode(lib, q=None) == 1
+    assert _decode(lib, num_pages=0) == 1
+    assert _decode(lib, num_pages=1 << 26) == 1          # 64 * pages must fit int32 rows
+    assert _decode(lib, max_pages=4) == 1                # stride smaller than max_pages
+    assert _decode(lib, q=(1 << 20) + 8) == 1            # misaligned q
+    assert _decode(lib, ws_bytes=16) == 5                # workspace too small
+    assert _decode(lib, ws=None) == 5
+    assert _decode(lib, scale=float("nan")) == 1
+
+
+def test_block_table_and_planner_validation():
+    lib = mla.library()
+    bt = lib.mla_build_block_table
+    ok = dict(r2t=1 << 20, rows=5, stride=192, rpi=1 << 21, rpi_dt=3, sl=1 << 22, sl_dt=2, add=0,
+              bs=2, out=1 << 23, out_stride=3, max_pages=3, page=64, fill=1, stream=None)
+    assert bt(*{**ok, "bs": 0}.values()) == 0
+    assert bt(*{**ok, "page": 16}.values()) == 1
+    assert bt(*{**ok, "rpi_dt": 0}.values()) == 1
+    assert bt(*{**ok, "out_stride": 2}.values()) == 1
+    assert bt(*{**ok, "r2t": None}.values()) == 1
+    md = lib.mla_get_mla_metadata
+    assert md(1 << 20, 2, 0, 0, 1 << 21, 1 << 22, None) == 1
+    assert md(1 << 20, -1, 74, 0, 1 << 21, 1 << 22, None) == 1
+    assert md(1 << 20, 2, 74, 0, (1 << 21) + 4, 1 << 22, None) == 1   # misaligned rows
