@@ -212,6 +212,43 @@ MLA_API mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs
  */
 MLA_API mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t stream);
 
+/*
+ * mla_decode_paged without a caller-supplied workspace.
+ *
+ * The pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory at the point where they run attention: an engine that plans
+ * every byte of device memory ahead of time and forbids allocation afterwards, a plugin
+ * whose host framework owns all device memory and rejects cudaMalloc inside its
+ * execute hook, or code running where cudaMalloc would block on the device or fail under
+ * memory pressure.  Such callers still pass every input and output buffer; only the
+ * split-KV scratch comes from the library.
+ *
+ * That scratch is one fixed array of MLA_NOALLOC_SCRATCH_BYTES (64 MiB) in the library's
+ * device memory.  Every GPU on which the library's kernels are loaded holds it until the
+ * process exits.  A problem whose workspace (mla_decode_workspace_bytes) exceeds it is
+ * rejected with MLA_ERR_WORKSPACE before anything is launched; the five DeepSeek-V3-shaped
+ * workloads of this project (up to bs 128 x 128 heads, or bs 32 x 4 x 128 rows) fit.
+ *
+ * All calls share the one array and it keeps whatever the last call left in it; the
+ * kernels write every scratch value before reading it, so nothing needs clearing.  Calls
+ * whose execution overlaps on the GPU (on different streams, or from different threads)
+ * race on the array and corrupt each other's results: serialise them.
+ *
+ * The first call on a device looks up the array's device address there (a host-side
+ * query, once per device, with that device current); make that first call before any
+ * stream capture.  This call allocates nothing: no cudaMalloc, no cudaFree.
+ * Arguments, results and errors are otherwise those of mla_decode_paged.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+MLA_API mla_status_t mla_decode_paged_noalloc(
+    const void* q, int32_t q_dtype, int32_t bs, int32_t q_len, int32_t h_q, int32_t head_dim,
+    int32_t head_dim_v, const void* k_cache, int32_t kv_dtype, int64_t num_pages,
+    int32_t page_size, const int32_t* block_table, int64_t block_table_stride, int32_t max_pages,
+    const int32_t* cache_seqlens, const int32_t* tile_scheduler_metadata, int32_t num_sm_parts,
+    const int32_t* num_splits, float softmax_scale, int32_t causal, const float* descale_q,
+    const float* descale_k, void* out, float* lse, mla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -243,3 +243,54 @@ mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Workspace-free variant of mla_decode_paged for callers that cannot allocate device
+// memory (see the header).  Its split-KV scratch is this fixed array, which every GPU
+// that loads the library holds until exit.
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+// The array's name is only a host-side stand-in; the device address must be looked up on
+// each device, with that device current.  Done once per device, on its first call.
+mla_status_t noalloc_scratch_address(void** out) {
+    static std::once_flag flags[kMaxDevices];
+    static void* addrs[kMaxDevices];
+    static cudaError_t results[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    std::call_once(flags[dev], [dev] {
+        void* p = nullptr;
+        results[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        addrs[dev] = p;
+    });
+    if (results[dev] != cudaSuccess || addrs[dev] == nullptr) return MLA_ERR_CUDA;
+    *out = addrs[dev];
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status_t mla_decode_paged_noalloc(
+    const void* q, int32_t q_dtype, int32_t bs, int32_t q_len, int32_t h_q, int32_t head_dim,
+    int32_t head_dim_v, const void* k_cache, int32_t kv_dtype, int64_t num_pages,
+    int32_t page_size, const int32_t* block_table, int64_t block_table_stride, int32_t max_pages,
+    const int32_t* cache_seqlens, const int32_t* tile_scheduler_metadata, int32_t num_sm_parts,
+    const int32_t* num_splits, float softmax_scale, int32_t causal, const float* descale_q,
+    const float* descale_k, void* out, float* lse, mla_stream_t stream) {
+    if (bs > 0 && q_len > 0 && h_q > 0 && num_sm_parts > 0 &&
+        mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts) > MLA_NOALLOC_SCRATCH_BYTES)
+        return MLA_ERR_WORKSPACE;  // the problem needs more scratch than the fixed array holds
+    void* scratch = nullptr;
+    if (bs > 0) {
+        const mla_status_t st = noalloc_scratch_address(&scratch);
+        if (st != MLA_OK) return st;
+    }
+    return mla_decode_paged(q, q_dtype, bs, q_len, h_q, head_dim, head_dim_v, k_cache, kv_dtype,
+                            num_pages, page_size, block_table, block_table_stride, max_pages,
+                            cache_seqlens, tile_scheduler_metadata, num_sm_parts, num_splits,
+                            softmax_scale, causal, descale_q, descale_k, out, lse, scratch,
+                            MLA_NOALLOC_SCRATCH_BYTES, stream);
+}
