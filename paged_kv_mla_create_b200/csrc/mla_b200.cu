@@ -174,25 +174,54 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     EncodeTiledFn encode = encode_tiled();
     if (!encode) return MLA_ERR_CUDA;
 
-    // KV pool as a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16, 64 x 64 boxes with
-    // 128-byte swizzle; rows past the end read as zeros.
-    CUtensorMap kv_map;
-    std::memset(&kv_map, 0, sizeof kv_map);
-    const cuuint64_t gdim[2] = {576, (cuuint64_t)num_pages * 64};
-    const cuuint64_t gstride[1] = {576 * 2};
-    const cuuint32_t box[2] = {64, 64};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult cr = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache),
-                         gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return MLA_ERR_CUDA;
-
+    // Tensor maps (bf16, 128-byte swizzle; coordinates past an extent read as zeros).  Each
+    // view orders its dimensions so that one load lands as consecutive 64-row x 64-column
+    // boxes (8 KB each), the layout the MMAs read:
+    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = 3 chunks of
+    //      one page (24 KB).
+    //   V: (64 columns, pool rows [1152 B], 2 column chunks [128 B], 4 blocks of 128 columns
+    //      [256 B]); a load = one CTA's 128 columns of a 256-output block of one page (16 KB).
+    //   Q: (64 columns, rows of a request [1152 B], 9 column chunks [128 B], requests); a load
+    //      = 64 query rows x 576 columns (72 KB).
     const int32_t rows = q_len * h_q;
+    CUtensorMap k_map, v_map, q_map;
+    std::memset(&k_map, 0, sizeof k_map);
+    std::memset(&v_map, 0, sizeof v_map);
+    std::memset(&q_map, 0, sizeof q_map);
+    const cuuint64_t pool_rows = (cuuint64_t)num_pages * 64;
+    {
+        const cuuint64_t gdim[3] = {64, pool_rows, 9};
+        const cuuint64_t gstride[2] = {1152, 128};
+        const cuuint32_t box[3] = {64, 64, 3};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), gdim, gstride,
+                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[4] = {64, pool_rows, 2, 4};
+        const cuuint64_t gstride[3] = {1152, 128, 256};
+        const cuuint32_t box[4] = {64, 64, 2, 1};
+        const cuuint32_t estride[4] = {1, 1, 1, 1};
+        if (encode(&v_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache), gdim, gstride,
+                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)bs};
+        const cuuint64_t gstride[3] = {1152, 128, (cuuint64_t)rows * 1152};
+        const cuuint32_t box[4] = {64, 64, 9, 1};
+        const cuuint32_t estride[4] = {1, 1, 1, 1};
+        if (encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), gdim, gstride, box,
+                   estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
+
     const size_t splits = (size_t)bs + (size_t)num_sm_parts;
     mla::decode::Params p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.kv_fp8 = nullptr;
     p.block_table = block_table;
     p.bt_stride = block_table_stride;
     p.max_pages = max_pages;
@@ -217,7 +246,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
     mla::decode::mla_decode_kernel<false><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
-        kv_map, p);
+        k_map, v_map, q_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     const dim3 cgrid((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
@@ -294,3 +323,11 @@ extern "C" mla_status_t mla_decode_paged_noalloc(
                             softmax_scale, causal, descale_q, descale_k, out, lse, scratch,
                             MLA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+#ifdef MLA_TRACE
+// Trace builds only: copy the pipeline trace to the host.
+extern "C" __attribute__((visibility("default"))) int mla_trace_dump(void* host, size_t bytes) {
+    if (bytes > sizeof(mla::decode::g_trace)) bytes = sizeof(mla::decode::g_trace);
+    return (int)cudaMemcpyFromSymbol(host, mla::decode::g_trace, bytes);
+}
+#endif
