@@ -69,7 +69,8 @@ enum {
     MLA_DEVERR_ROW_OUT_OF_RANGE = 2,   /* req_pool_indices[b] not a row of req_to_token: row skipped   */
     MLA_DEVERR_LEN_OUT_OF_RANGE = 4,   /* a length exceeds the table / req_to_token width: clamped     */
     MLA_DEVERR_BAD_METADATA = 8,       /* a scheduler row is not a valid cursor range: part skipped    */
-    MLA_DEVERR_WAIT_TIMEOUT = 16       /* a pipeline wait exceeded its bound: the CTA gave up          */
+    MLA_DEVERR_WAIT_TIMEOUT = 16,      /* a pipeline wait exceeded its bound: the CTA gave up          */
+    MLA_DEVERR_Q_RANGE = 32            /* e4m3 cache: a q value beyond the f16 range (|q| > 65504)     */
 };
 
 typedef struct CUstream_st* mla_stream_t;  /* identical to cudaStream_t */
@@ -168,6 +169,10 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *   v_j = k_j[0:512];  s_j = softmax_scale * descale_q * <q[b,i,h,:], k_j>;
  *   lse = ln sum_j exp(s_j);  o = sum_j exp(s_j - lse) v_j.
  *   A row with no allowed key gets o = 0 and lse = -inf.
+ *   Arithmetic: S in fp32 from bf16 products (bf16 cache) or f16 products (e4m3 cache:
+ *   e4m3 values and bf16 q values are exact in f16, so q must lie within f16's range,
+ *   |q| <= 65504, or MLA_DEVERR_Q_RANGE is recorded and o is undefined); P rounded to
+ *   bf16 (f16 with an e4m3 cache) for the P V product; O accumulated in fp32.
  *
  *   q                 bf16 [bs, q_len, h_q, head_dim], contiguous
  *   q_dtype           MLA_DTYPE_BF16

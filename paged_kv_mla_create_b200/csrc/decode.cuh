@@ -9,29 +9,34 @@
 //     row, so S = Q K^T and O = P V are dense tensor-core contractions.  In a pair MMA of
 //     M = 128 each CTA holds 64 rows: CTA r owns query rows [64r, 64r + 64).  Its half of
 //     an accumulator D[64 rows, N] lies in its tensor memory as 128 lanes x N/2 columns:
-//     lane l < 64 is row l for columns [0, N/2), lane 64 + l is row l for [N/2, N).
-//   * S tiles are 128 tokens = two pages.  For S the B operand is split along N, so CTA r
-//     loads page r of the tile (all 576 columns, in 64-column chunks); for O += P V the
-//     B operand (V, the first 512 columns of the same rows) is split along N = output
-//     columns: two N = 256 MMAs cover the 512 outputs and CTA r loads both pages'
-//     columns {256n + 128r + [0, 128)}, n = 0, 1 (a second, L2-served read of those
-//     bytes).  No data crosses distributed shared memory: the pair's tensor cores share
-//     their operands.  (Pair MMAs keep the tensor pipe busy only with N = 256: at N = 128
-//     each SM's half is 64 columns wide and runs at about half rate.)
+//     lane l < 64 is row l for columns [0, N/2), lane 64 + l is row l for [N/2, N).  An A
+//     operand read from tensor memory is read the same way: row l from lane l for D's
+//     columns [0, N/2) and from lane 64 + l for [N/2, N), two bf16 of consecutive k per
+//     32-bit column.
+//   * S tiles are 128 tokens = two pages.  For S the B operand is split along N (tokens):
+//     CTA r loads page r of the tile, all 576 columns, into a 72 KB slot (nine 64-column
+//     chunks; chunk c at 8 KB * c).  For O += P V the B operand (V, the first 512 columns)
+//     is split along N = output columns: in the MMA for output block n (256 columns) and
+//     page p, CTA 0 supplies columns 256n + [0, 128) (chunks 4n, 4n + 1) and CTA 1
+//     columns 256n + [128, 256) (chunks 4n + 2, 4n + 3) of page p, both at slot offset
+//     8 KB * (4n + 2p).  CTA p has its own page's chunks there already; the other CTA's
+//     chunks at that offset belong to its own page and are dead once S is computed, so
+//     after the S MMAs it loads the partner page's four chunks it needs (32 KB, an L2 hit:
+//     the partner CTA has just loaded that page) into exactly those positions.  Each KV
+//     byte crosses HBM once; each CTA takes in 72 + 32 KB per tile.
 //   * Tensor memory per CTA: S double buffer 2 x 64 columns, O 256 columns (64 rows x 512
-//     outputs).  Q (own 64 rows x 576, 72 KB) and P (64 rows x 128 tokens) live in shared
-//     memory; K streams through a 3-slot ring of 24 KB loads (three 64-column chunks of
-//     the CTA's page, warp 0) and V through a 4-slot ring of 16 KB loads (this CTA's 128
-//     columns of one 256-output block of one page, warp 2).  Loads are few and large because the TMA unit's cost is per
-//     load: 64 x 64 boxes stream at about 60% of HBM bandwidth, 24 KB loads at full rate.
-//   * Roles per CTA: warps 0 / 3 (Q, K) and 2 / 8 (V) TMA producers (page ids from the block
-//     table), warp 9 idle;
-//     warp 1 lane 0 of the leader issues every MMA; warps 4..7 (thread t = TMEM lane t:
-//     row t % 64, token half t / 64) run the online softmax: partner threads t and t ^ 64
-//     agree on each row's maximum through shared memory (an mbarrier orders the exchange,
-//     so a timed-out wait can never strand the others), P goes to shared memory for the
-//     PV MMA, O is rescaled in tensor memory only when the running maximum grows by more
-//     than 2^8, and the epilogue normalises and writes o and lse.
+//     outputs), and Q columns [0, 256) of the CTA's 64 rows (128 columns; row r in lanes r
+//     and 64 + r) as the A operand of the first four chunks of S; Q columns [256, 576) (40 KB) and P (64
+//     rows x 128 tokens, 16 KB) live in shared memory, with a 2-slot K ring (144 KB).
+//   * Roles per CTA: warps 0 / 3 load K (alternate tiles, one 72 KB load each), warp 2 the
+//     partner V after each tile's S, warps 8..11 load Q once per unit (columns [256, 576) by
+//     TMA into shared memory, columns [0, 256) into tensor memory) and prefetch the later
+//     units' query rows into L2; warp 1 lane 0 of the leader issues every MMA; warps 4..7 (thread t = TMEM lane t: row t % 64, token half
+//     t / 64) run the online softmax: partner threads t and t ^ 64 agree on each row's
+//     maximum through shared memory (an mbarrier orders the exchange, so a timed-out wait
+//     can never strand the others), P goes to shared memory for the PV MMA, O is rescaled
+//     in tensor memory only when the running maximum grows by more than 2^8, and the
+//     epilogue normalises and writes o and lse.
 //   * A unit whose block range is a whole request writes bf16 o and lse directly; a split
 //     piece writes fp32 partials that combine_splits_kernel merges.
 //   * Every wait is bounded (mbar_wait_bounded); out-of-range page ids never fault: TMA
@@ -66,39 +71,39 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kChunks = kDqk / 64;         // 64-column chunks of the 576 reduction columns
 constexpr int kBox = 64 * 128;             // one 64-row x 64-column bf16 box, 128-byte swizzle
-constexpr int kQBytes = kChunks * kBox;    // 72 KB: own 64 query rows
-constexpr int kKOpChunks = 3;             // one K load = 3 column chunks of the CTA's page (24 KB)
-constexpr int kKOps = kChunks / kKOpChunks;
-constexpr int kKSlots = 3;                 // K ring: one tile of K in flight per CTA
-constexpr int kKSlotBytes = kKOpChunks * kBox;
-constexpr int kVOps = 4;                   // per tile: (outputs 0-255, page 0), (0-255, page 1), (256-511, 0), (256-511, 1)
-constexpr int kVSlots = 4;                 // V ring: one tile of V
-constexpr int kVSlotBytes = 2 * kBox;      // one page x this CTA's 128 columns of a 256-output block
-constexpr int kPBytes = 2 * kBox;          // P: 64 rows x 128 tokens bf16 (single buffer)
-constexpr int kThreads = 320;              // 10 warps (roles below)
+constexpr int kQLoChunks = 4;              // Q columns [0, 256): tensor memory
+constexpr int kQHiChunks = kChunks - kQLoChunks;   // Q columns [256, 576): shared memory
+constexpr int kQHiBytes = kQHiChunks * kBox;       // 40 KB
+constexpr int kKSlots = 2;                 // K ring: two tiles
+constexpr int kKSlotBytes = kChunks * kBox;        // 72 KB: one page, all 576 columns
+constexpr int kVLoadBytes = 2 * kBox;      // one partner-V load: two chunks of one page
+constexpr int kPBytes = 2 * kBox;          // P: 64 rows x 128 tokens bf16
+constexpr int kThreads = 384;              // 12 warps (roles above)
 constexpr int kSoftmaxWarp0 = 4;
+constexpr int kQWarp0 = 8;                 // warps 8..11: Q loaders (TMEM lane quarters 0..3)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 // Tensor-memory column map (512 columns allocated for the pair).
 constexpr uint32_t kTmemS = 0;             // 2 x 64 columns
 constexpr uint32_t kTmemO = 128;           // 256 columns: block n (128 columns) holds outputs
                                            // 256n + [0, 128) in lanes < 64, 256n + 128 + [0, 128) above
+constexpr uint32_t kTmemQ = 384;           // 128 columns, lanes 0..63: Q columns 2j, 2j + 1 in column j
 constexpr uint32_t kTmemCols = 512;
 
 // Shared-memory map (offsets from the 1024-aligned base).
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKSlots * kKSlotBytes;
-constexpr int kOffP = kOffV + kVSlots * kVSlotBytes;
-constexpr int kOffX = kOffP + kPBytes;          // row-max exchange: 2 x 128 floats, row sums 128
+constexpr int kOffQ = 0;                            // Q chunks 4..8
+constexpr int kOffK = kOffQ + kQHiBytes;
+constexpr int kOffP = kOffK + kKSlots * kKSlotBytes;
+constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128 floats, row sums 128
 constexpr int kOffBar = kOffX + 3 * 128 * 4;
 
 enum : int {
-    kBarKFull = 0,                      // leader: both CTAs' K op landed (tx bytes)
-    kBarKEmpty = kBarKFull + kKSlots,   // both: pair MMAs finished reading a K slot
-    kBarVFull = kBarKEmpty + kKSlots,
-    kBarVEmpty = kBarVFull + kVSlots,
-    kBarQFull = kBarVEmpty + kVSlots,   // leader: both Q halves landed
+    kBarKFull = 0,                      // leader: both CTAs' pages landed (tx bytes)
+    kBarKEmpty = kBarKFull + kKSlots,   // both: the tile's PV MMAs finished (slot reusable)
+    kBarQKDone = kBarKEmpty + kKSlots,  // both: the tile's S MMAs finished reading the slot
+    kBarVFull = kBarQKDone + kKSlots,   // leader: both CTAs' partner V landed (tx bytes)
+    kBarQFull = kBarVFull + kKSlots,    // leader: Q columns [256, 576) landed (tx) + eight
+                                        // warps wrote Q columns [0, 256) to tensor memory
     kBarQEmpty,                         // both: the unit's last S MMA finished (Q reusable)
     kBarSFull,                          // both (x2): S tile in tensor memory
     kBarSFree = kBarSFull + 2,          // leader (x2): 8 softmax warps have read S
@@ -108,16 +113,58 @@ enum : int {
     kBarOEmpty,                         // leader: 8 softmax warps read O out
     kBarXchg,                           // local (x2): the 128 softmax threads posted row maxima
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
-    kNumBars
+    kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
+    kBarVRaw = kBarKRaw + kKSlots,      // local (x2), e4m3 cache: this CTA's partner V landed
+    kNumBars = kBarVRaw + kKSlots
 };
 
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
+constexpr uint32_t kIdescQK16 = idesc_bf16_f32(128, 128, false, false, true);
+constexpr uint32_t kIdescPV16 = idesc_bf16_f32(128, 256, false, true, true);
+
+// e4m3 cache: a page (64 rows x 576 one-byte values, 36 KB) lands in the back half of its
+// slot as nine 64 x 64-byte chunks and is widened in place, chunk by chunk from the front,
+// to the f16 layout of the bf16 path (chunk c at 8 KB * c): chunk c's output never reaches
+// the input of a chunk after c, and each chunk is read whole before it is written.
+constexpr int kPage8Bytes = kPage * kDqk;              // 36 KB
+constexpr int kRaw8Off = kKSlotBytes - kPage8Bytes;    // 36 KB into the slot
+constexpr int kChunk8 = 64 * 64;                       // one 64-row x 64-byte e4m3 chunk
+
+// Widen one e4m3 chunk (64 rows x 64 bytes at src) to f16 (64 rows x 128 bytes at dst,
+// 128-byte swizzle: 16-byte unit u of row t at u ^ (t & 7)).  One warp; the whole chunk
+// is read before any of it is written.
+__device__ __forceinline__ void widen_chunk_e4m3(uint32_t src, uint32_t dst, int lane) {
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = ld_shared_v4u(src + 16u * (uint32_t)(lane + 32 * j));
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int x = lane + 32 * j;        // row x / 4, 16-value quarter x % 4
+        const uint32_t t = (uint32_t)(x >> 2), q = (uint32_t)(x & 3);
+        const uint32_t row = dst + 128u * t;
+        st_shared_v4u(row + 16u * ((2u * q) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].x), e4m3x2_to_f16x2(v[j].x >> 16),
+                      e4m3x2_to_f16x2(v[j].y), e4m3x2_to_f16x2(v[j].y >> 16));
+        st_shared_v4u(row + 16u * ((2u * q + 1u) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].z),
+                      e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w), e4m3x2_to_f16x2(v[j].w >> 16));
+    }
+    __syncwarp();
+}
+
+// bf16 pair -> f16 pair (the e4m3 path computes in f16); flags values beyond f16's range.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& out_of_range) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    out_of_range |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+    return pack_f16x2(lo, hi);
+}
 
 struct Params {
+    const __nv_bfloat16* q;        // [bs, rows, 576]
     const int32_t* block_table;    // [bs, bt_stride]
     int64_t bt_stride;
     int32_t max_pages;
@@ -180,6 +227,41 @@ __device__ __forceinline__ UnitIter make_iter(const Params& p, int part, bool& o
 
 __device__ __forceinline__ int tiles_of(int kb0, int kb1) { return (kb1 - kb0 + 1) >> 1; }
 
+// Page ids of one unit's blocks for a whole warp: lanes hold blocks [base, base + 32), slid
+// forward as the tiles advance.  row(blk) is the TMA row coordinate page * 64, or the first
+// row past the pool (read as zeros) for a block past the unit or a bad page id.
+struct PageWindow {
+    const int32_t* bt_row;
+    int kb1, base, lane, pg;
+    int64_t num_pages;
+    bool report;
+    __device__ int fetch(int idx) {
+        const int v = idx < kb1 ? __ldg(bt_row + idx) : -1;
+        const bool bad = idx < kb1 && (v < 0 || (int64_t)v >= num_pages);
+        if (__any_sync(0xffffffffu, bad) && lane == 0 && report) raise_error(1 /* MLA_DEVERR_PAGE_OUT_OF_RANGE */);
+        return (idx < kb1 && !bad) ? v : -1;
+    }
+    __device__ void init(const int32_t* row, int kb0_, int kb1_, int lane_, int64_t np, bool rep) {
+        bt_row = row;
+        kb1 = kb1_;
+        base = kb0_;
+        lane = lane_;
+        num_pages = np;
+        report = rep;
+        pg = fetch(base + lane);
+    }
+    __device__ int32_t row(int blk) {
+        const int32_t past = (int32_t)(num_pages * kPage);
+        if (blk >= kb1) return past;
+        while (blk >= base + 32) {
+            base += 32;
+            pg = fetch(base + lane);
+        }
+        const int v = __shfl_sync(0xffffffffu, pg, blk - base);
+        return v >= 0 ? v * kPage : past;
+    }
+};
+
 template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
@@ -201,14 +283,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
-            mbar_init(bar(kBarKFull + s), 1);
+            // bf16: one arrival + the pair's TMA bytes; e4m3: each CTA's widening warp arrives
+            mbar_init(bar(kBarKFull + s), kFp8 ? 2 : 1);
             mbar_init(bar(kBarKEmpty + s), 1);
+            mbar_init(bar(kBarQKDone + s), 1);
+            mbar_init(bar(kBarVFull + s), kFp8 ? 2 : 1);
+            mbar_init(bar(kBarKRaw + s), 1);
+            mbar_init(bar(kBarVRaw + s), 1);
         }
-        for (int s = 0; s < kVSlots; ++s) {
-            mbar_init(bar(kBarVFull + s), 1);
-            mbar_init(bar(kBarVEmpty + s), 1);
-        }
-        mbar_init(bar(kBarQFull), 1);
+        // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
+        mbar_init(bar(kBarQFull), kFp8 ? 8 : 1 + 8);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
@@ -243,96 +327,77 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     UnitIter iter = make_iter(p, part, md_ok);
     if (!md_ok && threadIdx.x == 0) raise_error(8 /* MLA_DEVERR_BAD_METADATA */);
 
-    if (warp == 0 || warp == 2 || warp == 3 || warp == 8) {
-        // ------------------------------------------------------------ TMA producers
-        // A thread's TMA loads complete one after another (about 500 cycles plus 11 per KB
-        // each), so each stream has two issuing warps taking alternate loads: warps 0 / 3
-        // load Q (warp 0, once per unit) and K, three 24 KB loads per tile (three 64-column
-        // chunks of the CTA's page); warps 2 / 8 load V, four 16 KB loads per tile (this
-        // CTA's 128 columns 256n + 128r + [0, 128) of one page, in the order (n, page) =
-        // (0,0), (0,1), (1,0), (1,1) the PV MMAs consume).
-        const bool is_k = warp == 0 || warp == 3;
-        const uint32_t parity = (warp == 3 || warp == 8) ? 1u : 0u;
-        uint32_t oc = 0, uq = 0;   // this stream's load counter, unit counter
+    // Signals to the leader's barriers: the leader's own warps arrive locally; the peer's
+    // warps arrive remotely, releasing at cluster scope only when they publish data.
+    auto arrive_leader = [&](int b_idx) {
+        __syncwarp();
+        if (lane == 0) {
+            if (leader)
+                mbar_arrive(bar(b_idx));
+            else
+                mbar_arrive_remote(map_to_cta(bar(b_idx), 0));
+        }
+    };
+    auto arrive_leader_done_reading = [&](int b_idx) {
+        __syncwarp();
+        if (lane == 0) {
+            if (leader)
+                mbar_arrive(bar(b_idx));
+            else
+                mbar_arrive_remote_relaxed(map_to_cta(bar(b_idx), 0));
+        }
+    };
+
+    if (warp == 0 || warp == 3) {
+        // ------------------------------------------------------------ K producers
+        // One 72 KB load per tile (this CTA's page, all 576 columns); a thread's TMA loads
+        // start one after another, so two warps take alternate tiles (and slots).
+        const uint32_t mine = warp == 3 ? 1u : 0u;
+        uint32_t g = 0;
         bool alive = true;
         int ub, kb0, kb1;
         while (alive && iter.next(ub, kb0, kb1)) {
             const int n = tiles_of(kb0, kb1);
             if (n <= 0) continue;
-            const int32_t* bt_row = p.block_table + (int64_t)ub * p.bt_stride;
-            if (is_k && parity == 0) {
+            PageWindow pw;
+            pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, warp == 0);
+            for (int i = 0; i < n; ++i, ++g) {
+                const int32_t row = pw.row(kb0 + 2 * i + (int)rank);
+                if ((g & 1u) != mine) continue;
                 int ok = 1;
+                const int s = (int)(g & 1u);
+                const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                 if (lane == 0) {
-                    if (uq > 0)
-                        ok = mbar_wait_bounded<false>(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag);
+                    ok = mbar_wait_bounded<false>(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, abort_flag);
                     if (ok) {
-                        if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQBytes);
-                        // own 64 query rows, all 9 column chunks, one load
-                        tma_load_4d_pair(sbase + kOffQ, &q_map, map_to_cta(bar(kBarQFull), 0), 0,
-                                         mtile * kRows + kCtaRows * (int32_t)rank, 0, ub);
-                    }
-                }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            }
-            // Page ids of blocks [pg_base, pg_base + 32) across the warp, slid forward as the
-            // tiles advance.  Block j -> TMA row coordinate page * 64; a bad or missing page
-            // -> the first row past the pool, read as zeros (and reported).
-            int pg_base = kb0;
-            auto fetch_pg = [&](int idx) -> int {
-                const int pg = idx < kb1 ? __ldg(bt_row + idx) : -1;
-                const bool bad = idx < kb1 && (pg < 0 || (int64_t)pg >= p.num_pages);
-                if (__any_sync(0xffffffffu, bad) && lane == 0 && is_k && parity == 0) raise_error(1);
-                return (idx < kb1 && !bad) ? pg : -1;
-            };
-            int pg_lane = fetch_pg(kb0 + lane);
-            auto page_row = [&](int blk) -> int32_t {
-                if (blk >= kb1) return (int32_t)(p.num_pages * kPage);
-                while (blk >= pg_base + 32) {
-                    pg_base += 32;
-                    pg_lane = fetch_pg(pg_base + lane);
-                }
-                const int pg = __shfl_sync(0xffffffffu, pg_lane, blk - pg_base);
-                return pg >= 0 ? pg * kPage : (int32_t)(p.num_pages * kPage);
-            };
-            const int per_tile = is_k ? kKOps : kVOps;
-            for (int i = 0; alive && i < n; ++i) {
-                const int blk0 = kb0 + 2 * i;
-                const int32_t row0 = page_row(blk0), row1 = page_row(blk0 + 1);
-                for (int op = 0; op < per_tile; ++op, ++oc) {
-                    if ((oc & 1u) != parity) continue;
-                    int ok = 1;
-                    if (lane == 0) {
-                        if (is_k) {
-                            const int s = oc % kKSlots;
-                            ok = mbar_wait_bounded<false>(bar(kBarKEmpty + s), ((oc / kKSlots) & 1u) ^ 1u,
-                                                          abort_flag);
-                            if (ok) {
-                                if (leader) mbar_arrive_expect_tx(bar(kBarKFull + s), 2 * kKSlotBytes);
-                                tma_load_3d_pair(sbase + kOffK + s * kKSlotBytes, &k_map,
-                                                 map_to_cta(bar(kBarKFull + s), 0), 0, rank ? row1 : row0,
-                                                 kKOpChunks * op);
-                                MLA_TRACE_EVENT(i, 12 + op);
-                            }
+                        if constexpr (kFp8) {
+                            mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
+                            tma_load_3d(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0);
                         } else {
-                            const int s = oc % kVSlots;
-                            ok = mbar_wait_bounded<false>(bar(kBarVEmpty + s), ((oc / kVSlots) & 1u) ^ 1u,
-                                                          abort_flag);
-                            if (ok) {
-                                if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * kVSlotBytes);
-                                tma_load_4d_pair(sbase + kOffV + s * kVSlotBytes, &v_map,
-                                                 map_to_cta(bar(kBarVFull + s), 0), 0, (op & 1) ? row1 : row0, 0,
-                                                 2 * (op >> 1) + (int32_t)rank);
-                                MLA_TRACE_EVENT(i, 18 + op);
-                            }
+                            if (leader) mbar_arrive_expect_tx(bar(kBarKFull + s), 2 * kKSlotBytes);
+                            tma_load_3d_pair(slot, &k_map, map_to_cta(bar(kBarKFull + s), 0), 0, row, 0);
                         }
+                        MLA_TRACE_EVENT(g, 12);
                     }
-                    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    alive = false;
+                    break;
+                }
+                if constexpr (kFp8) {
+                    // the whole warp widens the page in place, then signals the leader
+                    const bool landed = mbar_wait_bounded<false>(bar(kBarKRaw + s), (g >> 1) & 1u, abort_flag);
+                    if (!__all_sync(0xffffffffu, landed)) {
                         alive = false;
                         break;
                     }
+#pragma unroll 1
+                    for (int c = 0; c < kChunks; ++c)
+                        widen_chunk_e4m3(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
+                    fence_proxy_async_smem();
+                    arrive_leader(kBarKFull + s);
                 }
             }
-            ++uq;
         }
         if (lane == 0 && *abort_flag) {
             // let copies already issued land before shared memory can go away
@@ -340,92 +405,269 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             while (global_timer_ns() - t0 < 200000ull) {
             }
         }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ partner V producer
+        // After a tile's S MMAs, the four chunks of the partner page this CTA supplies to the
+        // PV MMAs (columns 256n + 128r + [0, 128), n = 0, 1) go into the slot positions
+        // 4n + 2(1 - r), + 1, which held this CTA's own, now dead, chunks.
+        uint32_t g = 0;
+        bool alive = true;
+        int ub, kb0, kb1;
+        while (alive && iter.next(ub, kb0, kb1)) {
+            const int n = tiles_of(kb0, kb1);
+            if (n <= 0) continue;
+            PageWindow pw;
+            pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, false);
+            for (int i = 0; i < n; ++i, ++g) {
+                const int32_t row = pw.row(kb0 + 2 * i + 1 - (int)rank);
+                int ok = 1;
+                const int s = (int)(g & 1u);
+                const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
+                if (lane == 0) {
+                    ok = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                    if (ok) {
+                        if constexpr (kFp8) {
+                            // e4m3 chunks land in the back half of their 16 KB target region
+                            mbar_arrive_expect_tx(bar(kBarVRaw + s), 2 * 2 * kChunk8);
+#pragma unroll
+                            for (int nn = 0; nn < 2; ++nn)
+                                tma_load_3d(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox + kBox, &v_map,
+                                            bar(kBarVRaw + s), 0, row, 4 * nn + 2 * (int)rank);
+                        } else {
+                            if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * 2 * kVLoadBytes);
+#pragma unroll
+                            for (int nn = 0; nn < 2; ++nn)
+                                tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
+                                                 map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
+                        }
+                        MLA_TRACE_EVENT(g, 18);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    alive = false;
+                    break;
+                }
+                if constexpr (kFp8) {
+                    const bool landed = mbar_wait_bounded<false>(bar(kBarVRaw + s), (g >> 1) & 1u, abort_flag);
+                    if (!__all_sync(0xffffffffu, landed)) {
+                        alive = false;
+                        break;
+                    }
+#pragma unroll 1
+                    for (int nn = 0; nn < 2; ++nn) {
+                        const uint32_t region = slot + (4 * nn + 2 * (1 - (int)rank)) * kBox;
+                        widen_chunk_e4m3(region + kBox, region, lane);
+                        widen_chunk_e4m3(region + kBox + kChunk8, region + kBox, lane);
+                    }
+                    fence_proxy_async_smem();
+                    arrive_leader(kBarVFull + s);
+                }
+            }
+        }
+        if (lane == 0 && *abort_flag) {
+            // let copies already issued land before shared memory can go away
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 200000ull) {
+            }
+        }
+    } else if (warp >= kQWarp0) {
+        // ------------------------------------------------------------ Q loaders
+        // Per unit, once the previous unit's last S MMA has finished: warp kQWarp0 + 3
+        // (lane 0) loads Q columns [256, 576) of the CTA's 64 rows by TMA, and the four warps
+        // write Q columns [0, 256) into tensor memory, thread = lane.  A pair MMA reads an A
+        // operand from tensor memory for output columns [0, N/2) in lanes 0..63 and for
+        // [N/2, N) in lanes 64..127, so each row lies twice: lane r and lane 64 + r.
+        // Warp kQWarp0 + 2 (lane 0) first prefetches the query rows of the part's later
+        // units into L2.
+        const int quarter = warp & 3;
+        const int rloc = (32 * quarter + lane) & 63;
+        const int rowg = mtile * kRows + kCtaRows * (int)rank + rloc;
+        const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        if (quarter == 2 && lane == 0) {
+            UnitIter pk = iter;
+            int nb, a0, a1;
+            bool first = true;
+            while (pk.next(nb, a0, a1)) {
+                if (tiles_of(a0, a1) <= 0) continue;
+                if (!first) {
+                    tma_prefetch_4d(&q_map, 0, mtile * kRows + kCtaRows * (int32_t)rank, 0, nb);
+                    tma_prefetch_4d(&q_map, 0, mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, nb);
+                }
+                first = false;
+            }
+        }
+        uint32_t uq = 0;
+        bool q_range = false;
+        int ub, kb0, kb1;
+        while (iter.next(ub, kb0, kb1)) {
+            if (tiles_of(kb0, kb1) <= 0) continue;
+            if (uq > 0 && !mbar_wait_bounded<false>(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
+            tc_fence_after();
+            if (!kFp8 && quarter == 3 && lane == 0) {
+                if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQHiBytes);
+                tma_load_4d_pair(sbase + kOffQ, &q_map, map_to_cta(bar(kBarQFull), 0), 0,
+                                 mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, ub);
+            }
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)ub * p.rows + rowg) * kDqk);
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                uint4 v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[k] = rowg < p.rows ? __ldg(src + 4 * c + k) : make_uint4(0, 0, 0, 0);
+                uint32_t w[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    w[4 * k] = v[k].x;
+                    w[4 * k + 1] = v[k].y;
+                    w[4 * k + 2] = v[k].z;
+                    w[4 * k + 3] = v[k].w;
+                }
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], q_range);
+                }
+                tmem_st16(tmem + lane_off + kTmemQ + 16u * c, w);
+            }
+            if constexpr (kFp8) {
+                // Q columns [256, 576) as f16 into shared memory (128-byte swizzle): lane
+                // quarters 0 / 1 take chunks 0..2 of them, quarters 2 / 3 chunks 3..4
+                const int c0 = quarter < 2 ? 0 : 3, c1 = quarter < 2 ? 3 : kQHiChunks;
+#pragma unroll 1
+                for (int cc = c0; cc < c1; ++cc) {
+                    const uint32_t qrow = sbase + kOffQ + cc * kBox + (uint32_t)rloc * 128u;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint4 v = rowg < p.rows ? __ldg(src + 32 + 8 * cc + u) : make_uint4(0, 0, 0, 0);
+                        st_shared_v4u(qrow + 16u * ((uint32_t)u ^ ((uint32_t)rloc & 7u)),
+                                      bf16x2_to_f16x2(v.x, q_range), bf16x2_to_f16x2(v.y, q_range),
+                                      bf16x2_to_f16x2(v.z, q_range), bf16x2_to_f16x2(v.w, q_range));
+                    }
+                }
+                fence_proxy_async_smem();
+                if (__any_sync(0xffffffffu, q_range) && lane == 0) raise_error(32 /* MLA_DEVERR_Q_RANGE */);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            arrive_leader(kBarQFull);
+            ++uq;
+        }
+        if (!kFp8 && quarter == 3 && lane == 0 && *abort_flag) {
+            // let a Q copy already issued land before shared memory can go away
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 200000ull) {
+            }
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader)
-        // Per unit: QK(0), QK(1), PV(0), QK(2), PV(1), ..., PV(last): S runs one tile ahead
-        // of PV so the tensor pipe computes S(t+1) while the softmax works on tile t.
+        // Two cursors walk the same tiles: S(t) = Q K^T and O += P(t) V(t).  Whichever is
+        // ready goes first, PV before S: a slot is only refilled after its tile's PV, so a
+        // PV that waits behind an S whose page is still in flight would stall the ring.
+        // S(t) waits for its page, its S buffer (the softmax read S(t - 2)) and, first in a
+        // unit, the unit's Q; PV(t) waits for P(t), the partner V of tile t and, first in a
+        // unit, the epilogue of the previous unit having read O.
         if (leader && lane == 0) {
-            uint32_t g = 0, uq = 0, kc = 0, vc = 0;
-            bool alive = true;
-            int ub, kb0, kb1;
-            auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-                if (!mbar_wait_bounded<true>(bar(kBarPFull), gg & 1u, abort_flag)) return false;
-                if (first && uq > 0 &&
-                    !mbar_wait_bounded<true>(bar(kBarOEmpty), (uq - 1) & 1u, abort_flag))
-                    return false;
-                tc_fence_after();
-                MLA_TRACE_EVENT(gg, 2);
-                const uint32_t pbuf = sbase + kOffP;
-#pragma unroll 1
-                for (int vop = 0; vop < kVOps; ++vop) {
-                    const int pp = vop & 1;
-                    const int s = vc % kVSlots;
-                    if (!mbar_wait_bounded<true>(bar(kBarVFull + s), (vc / kVSlots) & 1u, abort_flag))
-                        return false;
-                    MLA_TRACE_EVENT(gg, 22 + vop);
-                    tc_fence_after();
-                    const uint32_t vslot = sbase + kOffV + s * kVSlotBytes;
-                    const int nn = vop >> 1;   // output block: TMEM columns 128nn..
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_pair_ss(tmem + kTmemO + 128u * nn,
-                                    smem_desc_sw128(pbuf + pp * kBox + 32u * kk, 16, 1024),
-                                    smem_desc_sw128(vslot + 2048u * kk, kBox, 1024), kIdescPV,
-                                    (first && pp == 0 && kk == 0) ? 0u : 1u);
-                    tc_commit_pair(bar(kBarVEmpty + s));
-                    ++vc;
-                }
-                tc_commit_pair(bar(kBarPvDone));
-                return true;
-            };
-            while (alive && iter.next(ub, kb0, kb1)) {
-                const int n = tiles_of(kb0, kb1);
-                if (n <= 0) continue;
-                if (!mbar_wait_bounded<true>(bar(kBarQFull), uq & 1u, abort_flag)) break;
-                const uint32_t g0 = g;
-                for (int i = 0; alive && i < n; ++i) {
-                    const uint32_t sb = g & 1u;
-                    if (g >= 2 &&
-                        !mbar_wait_bounded<true>(bar(kBarSFree + sb), ((g >> 1) & 1u) ^ 1u, abort_flag)) {
-                        alive = false;
-                        break;
-                    }
-                    MLA_TRACE_EVENT(g, 1);
-#pragma unroll 1
-                    for (int j = 0; j < kKOps; ++j) {
-                        const int s = kc % kKSlots;
-                        if (!mbar_wait_bounded<true>(bar(kBarKFull + s), (kc / kKSlots) & 1u, abort_flag)) {
-                            alive = false;
-                            break;
+            struct Cursor {
+                UnitIter it;
+                int n, i;
+                uint32_t g, uq;
+                bool valid;
+                __device__ void next_unit() {
+                    int ub_, a_, b_;
+                    valid = false;
+                    while (it.next(ub_, a_, b_)) {
+                        n = tiles_of(a_, b_);
+                        if (n > 0) {
+                            i = 0;
+                            valid = true;
+                            return;
                         }
-                        MLA_TRACE_EVENT(g, 15 + j);
+                    }
+                }
+                __device__ void step() {
+                    ++g;
+                    if (++i == n) {
+                        ++uq;
+                        next_unit();
+                    }
+                }
+            };
+            Cursor cq, cp;
+            cq.it = iter;
+            cq.g = 0;
+            cq.uq = 0;
+            cq.next_unit();
+            cp = cq;
+            uint64_t t_idle = global_timer_ns();
+            while (cq.valid || cp.valid) {
+                bool did = false;
+                if (cp.valid && cp.g < cq.g) {
+                    const int s = (int)(cp.g & 1u);
+                    const bool first = cp.i == 0;
+                    if (mbar_try_wait_cluster(bar(kBarPFull), cp.g & 1u) &&
+                        mbar_try_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
+                        (!first || cp.uq == 0 || mbar_try_wait_cluster(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
                         tc_fence_after();
-                        const uint32_t kslot = sbase + kOffK + s * kKSlotBytes;
+                        MLA_TRACE_EVENT(cp.g, 2);
+                        const uint32_t pbuf = sbase + kOffP;
+                        const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
 #pragma unroll
-                        for (int c = 0; c < kKOpChunks; ++c) {
-                            const uint32_t qa = sbase + kOffQ + (kKOpChunks * j + c) * kBox;
-                            const uint32_t kb = kslot + c * kBox;
+                        for (int nn = 0; nn < 2; ++nn)
+#pragma unroll
+                            for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_pair_ss(tmem + kTmemO + 128u * nn,
+                                                smem_desc_sw128(pbuf + pp * kBox + 32u * kk, 16, 1024),
+                                                smem_desc_sw128(slot + (4 * nn + 2 * pp) * kBox + 2048u * kk, kBox, 1024),
+                                                kFp8 ? kIdescPV16 : kIdescPV, (first && pp == 0 && kk == 0) ? 0u : 1u);
+                        tc_commit_pair(bar(kBarKEmpty + s));
+                        tc_commit_pair(bar(kBarPvDone));
+                        if (cp.i == cp.n - 1) tc_commit_pair(bar(kBarOFull));
+                        cp.step();
+                        did = true;
+                    }
+                }
+                if (!did && cq.valid) {
+                    const int s = (int)(cq.g & 1u);
+                    const uint32_t sb = cq.g & 1u;
+                    if ((cq.i != 0 || mbar_try_wait_cluster(bar(kBarQFull), cq.uq & 1u)) &&
+                        (cq.g < 2 || mbar_try_wait_cluster(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
+                        mbar_try_wait_cluster(bar(kBarKFull + s), (cq.g >> 1) & 1u)) {
+                        tc_fence_after();
+                        MLA_TRACE_EVENT(cq.g, 15);
+                        const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
+                        const uint32_t d = tmem + kTmemS + 64u * sb;
+#pragma unroll
+                        for (int c = 0; c < kQLoChunks; ++c)
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                mma_pair_ss(tmem + kTmemS + 64u * sb, smem_desc_sw128(qa + 32u * kk, 16, 1024),
-                                            smem_desc_sw128(kb + 32u * kk, 16, 1024), kIdescQK,
-                                            (j | c | kk) ? 1u : 0u);
-                        }
-                        tc_commit_pair(bar(kBarKEmpty + s));
-                        ++kc;
+                                mma_pair_ts(d, tmem + kTmemQ + 32u * c + 8u * kk,
+                                            smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                            kFp8 ? kIdescQK16 : kIdescQK, (c | kk) ? 1u : 0u);
+#pragma unroll
+                        for (int c = kQLoChunks; c < kChunks; ++c)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_pair_ss(d, smem_desc_sw128(sbase + kOffQ + (c - kQLoChunks) * kBox + 32u * kk, 16, 1024),
+                                            smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                            kFp8 ? kIdescQK16 : kIdescQK, 1u);
+                        tc_commit_pair(bar(kBarQKDone + s));
+                        tc_commit_pair(bar(kBarSFull + sb));
+                        if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
+                        cq.step();
+                        did = true;
                     }
-                    if (!alive) break;
-                    tc_commit_pair(bar(kBarSFull + sb));
-                    if (i == n - 1) tc_commit_pair(bar(kBarQEmpty));
-                    if (i >= 1 && !issue_pv(g - 1, i == 1)) {
-                        alive = false;
+                }
+                if (did) {
+                    t_idle = global_timer_ns();
+                } else {
+                    if (*abort_flag) break;
+                    if (global_timer_ns() - t_idle > kWaitBudgetNs) {
+                        raise_error(16 /* MLA_DEVERR_WAIT_TIMEOUT */);
+                        *abort_flag = 1;
                         break;
                     }
-                    ++g;
                 }
-                if (!alive || !issue_pv(g - 1, g - 1 == g0)) break;
-                tc_commit_pair(bar(kBarOFull));
-                ++uq;
             }
         }
     } else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + 4) {
@@ -442,26 +684,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         const float sl2 = p.scale_log2 * dq * dk;
         float* xmax = reinterpret_cast<float*>(smem + kOffX);  // [2][128] row maxima, [128] sums
         const uint32_t swz = (uint32_t)(rloc & 7);
-        // Signals to the leader's barriers: the leader's own warps arrive locally; the peer's
-        // warps arrive remotely, releasing at cluster scope only when they publish data.
-        auto arrive_leader = [&](int b_idx) {
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(bar(b_idx));
-                else
-                    mbar_arrive_remote(map_to_cta(bar(b_idx), 0));
-            }
-        };
-        auto arrive_leader_done_reading = [&](int b_idx) {
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(bar(b_idx));
-                else
-                    mbar_arrive_remote_relaxed(map_to_cta(bar(b_idx), 0));
-            }
-        };
 
         auto write_empty = [&](int b) {
             // A request with no key: o = 0, lse = -inf (always a single, direct piece).
@@ -551,7 +773,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     const float p0 = live ? fast_exp2(s[2 * j] - m_run) : 0.f;
                     const float p1 = live ? fast_exp2(s[2 * j + 1] - m_run) : 0.f;
                     psum += p0 + p1;
-                    s[j] = __uint_as_float(pack_bf16x2(p0, p1));
+                    s[j] = __uint_as_float(kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1));
                 }
                 l_half += psum;
                 if (t == 0) MLA_TRACE_EVENT(g, 5);

@@ -56,6 +56,10 @@ mla_status_t prepare_decode_kernels() {
         results[dev] = cudaFuncSetAttribute(mla::decode::mla_decode_kernel<false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mla::decode::kSmemBytes);
+        if (results[dev] == cudaSuccess)
+            results[dev] = cudaFuncSetAttribute(mla::decode::mla_decode_kernel<true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                mla::decode::kSmemBytes);
     });
     return from_cuda(results[dev]);
 }
@@ -153,7 +157,6 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     if (head_dim != 576 || head_dim_v != 512 || page_size != 64) return MLA_ERR_UNSUPPORTED;
     if (q_dtype != MLA_DTYPE_BF16) return MLA_ERR_UNSUPPORTED;
     if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
-    if (kv_dtype == MLA_DTYPE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (bs == 0) return MLA_OK;
@@ -177,42 +180,53 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // Tensor maps (bf16, 128-byte swizzle; coordinates past an extent read as zeros).  Each
     // view orders its dimensions so that one load lands as consecutive 64-row x 64-column
     // boxes (8 KB each), the layout the MMAs read:
-    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = 3 chunks of
-    //      one page (24 KB).
-    //   V: (64 columns, pool rows [1152 B], 2 column chunks [128 B], 4 blocks of 128 columns
-    //      [256 B]); a load = one CTA's 128 columns of a 256-output block of one page (16 KB).
+    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = one page, all
+    //      576 columns (72 KB); also the box of the L2 prefetches.
+    //   V: the same view; a load = 2 column chunks of one page (16 KB).
     //   Q: (64 columns, rows of a request [1152 B], 9 column chunks [128 B], requests); a load
-    //      = 64 query rows x 576 columns (72 KB).
+    //      = 64 query rows x columns [256, 576) (40 KB).
     const int32_t rows = q_len * h_q;
     CUtensorMap k_map, v_map, q_map;
     std::memset(&k_map, 0, sizeof k_map);
     std::memset(&v_map, 0, sizeof v_map);
     std::memset(&q_map, 0, sizeof q_map);
     const cuuint64_t pool_rows = (cuuint64_t)num_pages * 64;
-    {
+    const bool fp8 = kv_dtype == MLA_DTYPE_FP8_E4M3;
+    if (!fp8) {
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {1152, 128};
-        const cuuint32_t box[3] = {64, 64, 3};
+        const cuuint32_t kbox[3] = {64, 64, 9};
+        const cuuint32_t vbox[3] = {64, 64, 2};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), gdim, gstride,
-                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   kbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MLA_ERR_CUDA;
-    }
-    {
-        const cuuint64_t gdim[4] = {64, pool_rows, 2, 4};
-        const cuuint64_t gstride[3] = {1152, 128, 256};
-        const cuuint32_t box[4] = {64, 64, 2, 1};
-        const cuuint32_t estride[4] = {1, 1, 1, 1};
-        if (encode(&v_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache), gdim, gstride,
-                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        if (encode(&v_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), gdim, gstride,
+                   vbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    } else {
+        // e4m3: (64 one-byte columns, pool rows [576 B], 9 column chunks [64 B]), no swizzle;
+        // a K load = one page as 9 chunks of 64 rows x 64 bytes (36 KB), a V load = 2 chunks.
+        const cuuint64_t gdim[3] = {64, pool_rows, 9};
+        const cuuint64_t gstride[2] = {576, 64};
+        const cuuint32_t kbox[3] = {64, 64, 9};
+        const cuuint32_t vbox[3] = {64, 64, 2};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(k_cache), gdim, gstride,
+                   kbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+        if (encode(&v_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(k_cache), gdim, gstride,
+                   vbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MLA_ERR_CUDA;
     }
     {
         const cuuint64_t gdim[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)bs};
         const cuuint64_t gstride[3] = {1152, 128, (cuuint64_t)rows * 1152};
-        const cuuint32_t box[4] = {64, 64, 9, 1};
+        const cuuint32_t box[4] = {64, 64, 5, 1};
         const cuuint32_t estride[4] = {1, 1, 1, 1};
         if (encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), gdim, gstride, box,
                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -222,6 +236,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
 
     const size_t splits = (size_t)bs + (size_t)num_sm_parts;
     mla::decode::Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
     p.block_table = block_table;
     p.bt_stride = block_table_stride;
     p.max_pages = max_pages;
@@ -245,8 +260,12 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
-    mla::decode::mla_decode_kernel<false><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
-        k_map, v_map, q_map, p);
+    if (fp8)
+        mla::decode::mla_decode_kernel<true><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
+            k_map, v_map, q_map, p);
+    else
+        mla::decode::mla_decode_kernel<false><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
+            k_map, v_map, q_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     const dim3 cgrid((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);

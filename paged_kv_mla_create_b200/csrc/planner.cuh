@@ -5,13 +5,20 @@
 //
 // The plan is a greedy balanced partition of 64-token blocks: every piece of a request
 // costs its blocks plus kFixedOverhead; total = sum_b (blocks_b + kFixedOverhead) and
-// each part gets the budget cdiv(total, parts) + kFixedOverhead, filled in request order.
-// A request that fits in what is left of the budget is taken whole; otherwise the part
-// takes (budget - kFixedOverhead) blocks of it when that is positive, and ends.
+// each part gets the budget P = cdiv(total, parts) + kFixedOverhead, filled in request
+// order.  A request that fits in what is left of the budget is taken whole; otherwise the
+// part takes (budget - kFixedOverhead) blocks of it when that is positive, and ends.
 //
-// One CTA: 256 threads stage the lengths in shared memory (as block counts) and reduce
-// the total; thread 0 then walks the parts, O(bs + parts) steps of a few instructions
-// each, with the next request's block count read one step ahead.
+// The walk is computed per request rather than per part: entering request b with r of
+// part i's budget left, either it fits (r >= blocks + F), or, after skipping to a fresh
+// part when r <= F, its first piece takes r - F blocks, the following parts take
+// Q = P - F blocks each, and the last piece takes the rest (1..Q blocks) -- a closed form
+// with one division.  One thread runs that O(bs) recurrence (each step a few
+// instructions, so a request costs what one part's step cost before); then one thread
+// per part reads its row off the per-request results by binary search: its first piece
+// belongs to the first request whose last part is >= i, its last to the last request
+// whose first part is <= i.  Batches larger than kPlannerSmemLens take the part-by-part
+// walk instead, reading the lengths from global memory.
 #pragma once
 #include "ptx.cuh"
 
@@ -19,88 +26,149 @@ namespace mla {
 
 constexpr int kFixedOverhead = 5;        // blocks of cost charged per piece
 constexpr int kPlannerThreads = 256;
-constexpr int kPlannerSmemLens = 8192;   // requests staged in shared memory (32 KB)
-constexpr int kPlannerSmemParts = 320;   // scheduler rows staged in shared memory (10 KB)
+constexpr int kPlannerSmemLens = 2048;   // requests handled by the per-request walk
 
 __global__ void __launch_bounds__(kPlannerThreads)
 get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, int32_t parts,
                         int32_t* __restrict__ md, int32_t* __restrict__ num_splits) {
-    // s_blocks[b] holds request b's block count until the walk passes it, then
-    // num_splits[b + 1] (the walk reads entry b before it writes it).
-    __shared__ int32_t s_blocks[kPlannerSmemLens + 1];
-    __shared__ int4 s_rows[kPlannerSmemParts * 2];
+    __shared__ int32_t s_nb[kPlannerSmemLens + 1];   // blocks of request b
+    __shared__ int32_t s_fp[kPlannerSmemLens];       // first part of request b
+    __shared__ int32_t s_lp[kPlannerSmemLens];       // last part of request b
+    __shared__ int32_t s_x0[kPlannerSmemLens];       // blocks of its first piece
+    __shared__ int32_t s_cum[kPlannerSmemLens];      // num_splits[b + 1]
     __shared__ long long s_warp_sum[kPlannerThreads / 32];
     const bool staged = bs <= kPlannerSmemLens;
-    const bool rows_staged = parts <= kPlannerSmemParts;
     long long local = 0;
     for (int b = threadIdx.x; b < bs; b += blockDim.x) {
         const int32_t L = cache_seqlens[b];
         const int32_t nb = L > 0 ? (L + 63) / 64 : 0;
-        if (staged) s_blocks[b] = nb;
+        if (staged) s_nb[b] = nb;
         local += nb + kFixedOverhead;
     }
-    if (staged && threadIdx.x == 0) s_blocks[bs] = 0;
+    if (staged && threadIdx.x == 0) s_nb[bs] = 0;
     for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xffffffffu, local, off);
     if ((threadIdx.x & 31) == 0) s_warp_sum[threadIdx.x >> 5] = local;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        long long total = 0;
+    long long total = 0;
 #pragma unroll
-        for (int w = 0; w < kPlannerThreads / 32; ++w) total += s_warp_sum[w];
-        // Budgets fit in 32 bits for any table a decode step can address (< 2^31 blocks).
-        const int payload = (int)((total + parts - 1) / parts) + kFixedOverhead;
-        auto blocks_of = [&](int b) -> int {
-            if (staged) return s_blocks[b];
-            if (b >= bs) return 0;
-            const int32_t L = cache_seqlens[b];
-            return L > 0 ? (L + 63) / 64 : 0;
-        };
-        int b = 0, k = 0, s = 0, cum = 0;
-        int nb = bs > 0 ? blocks_of(0) : 0;  // blocks of request b, read one step ahead
-        for (int i = 0; i < parts; ++i) {
-            const int begin_b = b, begin_k = k, begin_s = s;
-            int budget = payload;
-            while (b < bs) {
-                const int rem = nb - k;
-                if (budget >= rem + kFixedOverhead) {
-                    cum += s + 1;
-                    if (staged)
-                        s_blocks[b] = cum;
-                    else
+    for (int w = 0; w < kPlannerThreads / 32; ++w) total += s_warp_sum[w];
+    // Budgets fit in 32 bits for any table a decode step can address (< 2^31 blocks).
+    const int P = (int)((total + parts - 1) / parts) + kFixedOverhead;
+    const int Q = P - kFixedOverhead;   // >= 1
+
+    if (!staged) {
+        // part-by-part walk, lengths from global memory
+        if (threadIdx.x == 0) {
+            auto blocks_of = [&](int b) -> int {
+                if (b >= bs) return 0;
+                const int32_t L = cache_seqlens[b];
+                return L > 0 ? (L + 63) / 64 : 0;
+            };
+            num_splits[0] = 0;
+            int b = 0, k = 0, s = 0, cum = 0;
+            int nb = blocks_of(0);
+            for (int i = 0; i < parts; ++i) {
+                const int begin_b = b, begin_k = k, begin_s = s;
+                int budget = P;
+                while (b < bs) {
+                    const int rem = nb - k;
+                    if (budget >= rem + kFixedOverhead) {
+                        cum += s + 1;
                         num_splits[b + 1] = cum;
-                    budget -= rem + kFixedOverhead;
-                    ++b;
-                    nb = blocks_of(b);
-                    k = 0;
-                    s = 0;
-                } else {
-                    if (budget > kFixedOverhead) {
-                        k += budget - kFixedOverhead;
-                        ++s;
+                        budget -= rem + kFixedOverhead;
+                        ++b;
+                        nb = blocks_of(b);
+                        k = 0;
+                        s = 0;
+                    } else {
+                        if (budget > kFixedOverhead) {
+                            k += budget - kFixedOverhead;
+                            ++s;
+                        }
+                        break;
                     }
-                    break;
                 }
-            }
-            const int4 r0 = make_int4(begin_b, begin_k, b, k);
-            const int4 r1 = make_int4(begin_s, 0, 0, 0);
-            if (rows_staged) {
-                s_rows[2 * i] = r0;
-                s_rows[2 * i + 1] = r1;
-            } else {
                 int4* row = reinterpret_cast<int4*>(md + 8 * static_cast<int64_t>(i));
-                row[0] = r0;
-                row[1] = r1;
+                row[0] = make_int4(begin_b, begin_k, b, k);
+                row[1] = make_int4(begin_s, 0, 0, 0);
             }
+        }
+        return;
+    }
+
+    if (threadIdx.x == 0) {
+        int i = 0, r = P, cum = 0;
+        int nb = s_nb[0];
+        for (int b = 0; b < bs; ++b) {
+            const int nb_next = s_nb[b + 1];
+            const int c = nb + kFixedOverhead;
+            if (r < c && r <= kFixedOverhead) {   // the part ends with budget unused
+                ++i;
+                r = P;
+            }
+            int pieces, x0;
+            s_fp[b] = i;
+            if (r >= c) {
+                pieces = 1;
+                x0 = nb;
+                r -= c;
+            } else {
+                x0 = r - kFixedOverhead;          // 1 <= x0 < nb
+                const int rem = nb - x0;          // >= 1
+                const int m = (rem - 1) / Q;      // full middle pieces
+                const int last = rem - m * Q;     // 1..Q
+                pieces = 2 + m;
+                i += 1 + m;
+                r = P - last - kFixedOverhead;
+            }
+            s_lp[b] = i;
+            s_x0[b] = x0;
+            cum += pieces;
+            s_cum[b] = cum;
+            nb = nb_next;
         }
     }
     __syncthreads();
-    // coalesced write-back of what the walk staged
     if (threadIdx.x == 0) num_splits[0] = 0;
-    if (staged)
-        for (int b = threadIdx.x; b < bs; b += blockDim.x) num_splits[b + 1] = s_blocks[b];
-    if (rows_staged)
-        for (int i = threadIdx.x; i < 2 * parts; i += blockDim.x)
-            reinterpret_cast<int4*>(md)[i] = s_rows[i];
+    for (int b = threadIdx.x; b < bs; b += blockDim.x) num_splits[b + 1] = s_cum[b];
+    for (int i = threadIdx.x; i < parts; i += blockDim.x) {
+        int lo = 0, hi = bs;   // first request whose last part is >= i
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (s_lp[mid] >= i)
+                hi = mid;
+            else
+                lo = mid + 1;
+        }
+        const int bb = lo;
+        int4 r0 = make_int4(bs, 0, bs, 0), r1 = make_int4(0, 0, 0, 0);
+        if (bb < bs) {
+            int begin_k = 0, begin_s = 0;
+            if (s_fp[bb] < i) {   // the part starts inside request bb
+                begin_s = i - s_fp[bb];
+                begin_k = s_x0[bb] + (begin_s - 1) * Q;
+            }
+            int lo2 = bb, hi2 = bs;   // last request whose first part is <= i
+            while (lo2 < hi2) {
+                const int mid = (lo2 + hi2) >> 1;
+                if (s_fp[mid] <= i)
+                    lo2 = mid + 1;
+                else
+                    hi2 = mid;
+            }
+            const int bl = lo2 - 1;
+            int end_b = bl + 1, end_k = 0;
+            if (s_lp[bl] > i) {   // the part ends inside request bl
+                end_b = bl;
+                end_k = s_x0[bl] + (i - s_fp[bl]) * Q;
+            }
+            r0 = make_int4(bb, begin_k, end_b, end_k);
+            r1 = make_int4(begin_s, 0, 0, 0);
+        }
+        int4* row = reinterpret_cast<int4*>(md + 8 * static_cast<int64_t>(i));
+        row[0] = r0;
+        row[1] = r1;
+    }
 }
 
 }  // namespace mla

@@ -210,10 +210,10 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                       bool b_mn_major) {
+                                                       bool b_mn_major, bool f16 = false) {
     return (1u << 4)                              // D format: f32
-           | (1u << 7)                            // A format: bf16
-           | (1u << 10)                           // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)               // A format: bf16 (1) or f16 (0)
+           | ((f16 ? 0u : 1u) << 10)              // B format: bf16 (1) or f16 (0)
            | ((a_mn_major ? 1u : 0u) << 15)       // A major
            | ((b_mn_major ? 1u : 0u) << 16)       // B major
            | ((uint32_t)(N >> 3) << 17)           // N / 8
@@ -252,6 +252,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // ------------------------------------------------------------------ pair (cta_group::2)
+// TMA load into this CTA's shared memory, completing on this CTA's mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // TMA load whose bytes complete on an mbarrier of the pair's leader CTA (cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
                                                  uint32_t leader_bar, int32_t c0, int32_t c1) {
@@ -291,6 +301,14 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int32_t 
                  : "memory");
 }
 
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                int32_t c2, int32_t c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // Arrive on a peer CTA's mbarrier without ordering this thread's memory accesses (for
 // signals whose data dependence was already resolved, e.g. a completed tensor-memory read).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
@@ -325,6 +343,17 @@ __device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, ui
 
 // Arrive on `bar` (same offset) in both CTAs of the pair once the pair MMAs issued so far
 // have completed.
+// As mma_pair_ss with A read from tensor memory: each CTA's 64 rows of A in lanes 0..63
+// at columns a_tmem.., two bf16 of consecutive k per 32-bit column.
+__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
@@ -345,6 +374,28 @@ __device__ __forceinline__ void st_shared_v4u(uint32_t addr, uint32_t a, uint32_
 }
 
 // bf16x2 from two floats, round to nearest even; `lo` goes to the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two e4m3 values (first in the low byte) -> two f16 (first in the low half); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+    uint32_t r;
+    const uint16_t v = (uint16_t)two_bytes;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4u(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

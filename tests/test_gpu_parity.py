@@ -130,6 +130,18 @@ def test_non_causal_multi_query(mla):
     check_full(mla, wl)
 
 
+@pytest.mark.parametrize("lens,h,q_len", [([37, 130], 16, 1), ([1, 63, 64, 65, 127, 128, 129], 128, 1),
+                                         ([2000, 33, 700, 4000, 129], 128, 1), ([1000, 62, 129, 1], 128, 4)])
+def test_fp8_cache(mla, lens, h, q_len):
+    """e4m3 cache with a per-tensor scale; compared with the oracle on the same codes."""
+    check_full(mla, W.make_case(lens, h=h, q_len=q_len, kv="fp8", verify=q_len > 1, seed=31,
+                                poison=True))
+
+
+def test_fp8_cache_forced_splits(mla):
+    check_full(mla, W.make_case([2000, 33, 700, 4000, 129], h=128, kv="fp8", seed=32, poison=True), 7)
+
+
 def test_zero_length_request(mla):
     check_full(mla, W.make_case([0, 100, 0, 64], h=128, seed=26))
 
@@ -182,8 +194,6 @@ def sample_rows(wl, n, seed):
 @pytest.mark.parametrize("index", [2, 3, 4, 5])
 def test_full_size_workload_sampled(mla, index):
     wl = W.make_workload(index)
-    if wl.is_fp8:
-        pytest.skip("fp8 KV path not built yet")
     bt, md, ns, o, lse = run_path(mla, wl)
     check_metadata(mla, wl, bt, md, ns)
     rows = sample_rows(wl, 96 if index != 3 else 40, seed=index)
