@@ -22,16 +22,18 @@
 //     8 KB * (4n + 2p).  CTA p has its own page's chunks there already; the other CTA's
 //     chunks at that offset belong to its own page and are dead once S is computed, so
 //     after the S MMAs it loads the partner page's four chunks it needs (32 KB, an L2 hit:
-//     the partner CTA has just loaded that page) into exactly those positions.  Each KV
-//     byte crosses HBM once; each CTA takes in 72 + 32 KB per tile.
+//     the partner CTA loads that page) into exactly those positions.  Each KV byte crosses
+//     HBM once; each CTA takes in 72 + 32 KB per tile.
 //   * Tensor memory per CTA: S double buffer 2 x 64 columns, O 256 columns (64 rows x 512
 //     outputs), and Q columns [0, 256) of the CTA's 64 rows (128 columns; row r in lanes r
 //     and 64 + r) as the A operand of the first four chunks of S; Q columns [256, 576) (40 KB) and P (64
 //     rows x 128 tokens, 16 KB) live in shared memory, with a 2-slot K ring (144 KB).
-//   * Roles per CTA: warps 0 / 3 load K (alternate tiles, one 72 KB load each), warp 2 the
-//     partner V after each tile's S, warps 8..11 load Q once per unit (columns [256, 576) by
-//     TMA into shared memory, columns [0, 256) into tensor memory) and prefetch the later
-//     units' query rows into L2; warp 1 lane 0 of the leader issues every MMA; warps 4..7 (thread t = TMEM lane t: row t % 64, token half
+//   * Roles per CTA: warps 0 / 3 load K (alternate tiles, one 72 KB load each); warps 8..11
+//     load Q once per unit (columns [256, 576) by TMA into shared memory, columns [0, 256)
+//     into tensor memory), and warp 11 loads the partner V of every tile by TMA once the
+//     tile's S is done (an e4m3 cache: all four warps, through registers, widening to f16),
+//     and prefetch the later units' query rows into L2; warp 1 lane 0 of the leader issues
+//     every MMA; warps 4..7 (thread t = TMEM lane t: row t % 64, token half
 //     t / 64) run the online softmax: partner threads t and t ^ 64 agree on each row's
 //     maximum through shared memory (an mbarrier orders the exchange, so a timed-out wait
 //     can never strand the others), P goes to shared memory for the PV MMA, O is rescaled
@@ -76,7 +78,20 @@ constexpr int kQHiChunks = kChunks - kQLoChunks;   // Q columns [256, 576): shar
 constexpr int kQHiBytes = kQHiChunks * kBox;       // 40 KB
 constexpr int kKSlots = 2;                 // K ring: two tiles
 constexpr int kKSlotBytes = kChunks * kBox;        // 72 KB: one page, all 576 columns
-constexpr int kVLoadBytes = 2 * kBox;      // one partner-V load: two chunks of one page
+#ifndef MLA_KOPS
+#define MLA_KOPS 1
+#endif
+#ifndef MLA_V_TMA
+#define MLA_V_TMA 1
+#endif
+// Measured alternatives, kept selectable: the page loaded in three 24 KB pieces by three
+// warps (S starting on the first piece), and the bf16 partner V through registers like the
+// e4m3 one, were each slower on B200 than one 72 KB load and a TMA load of the partner V
+// (the SM's TMA unit and its global loads share one path; more, smaller requests cost more).
+constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
+constexpr int kKOpChunks = kChunks / kKOps;
+constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
+static_assert(kKOps == 1 || kKOps == 3, "page pieces");
 constexpr int kPBytes = 2 * kBox;          // P: 64 rows x 128 tokens bf16
 constexpr int kThreads = 384;              // 12 warps (roles above)
 constexpr int kSoftmaxWarp0 = 4;
@@ -98,10 +113,10 @@ constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128
 constexpr int kOffBar = kOffX + 3 * 128 * 4;
 
 enum : int {
-    kBarKFull = 0,                      // leader: both CTAs' pages landed (tx bytes)
-    kBarKEmpty = kBarKFull + kKSlots,   // both: the tile's PV MMAs finished (slot reusable)
+    kBarKFull = 0,                      // leader (x slots x pieces): both CTAs' piece j landed
+    kBarKEmpty = kBarKFull + kKSlots * kKOps,   // both: the tile's PV finished (slot reusable)
     kBarQKDone = kBarKEmpty + kKSlots,  // both: the tile's S MMAs finished reading the slot
-    kBarVFull = kBarQKDone + kKSlots,   // leader: both CTAs' partner V landed (tx bytes)
+    kBarVFull = kBarQKDone + kKSlots,   // leader: the 8 Q warps stored the partner V
     kBarQFull = kBarVFull + kKSlots,    // leader: Q columns [256, 576) landed (tx) + eight
                                         // warps wrote Q columns [0, 256) to tensor memory
     kBarQEmpty,                         // both: the unit's last S MMA finished (Q reusable)
@@ -114,8 +129,7 @@ enum : int {
     kBarXchg,                           // local (x2): the 128 softmax threads posted row maxima
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
-    kBarVRaw = kBarKRaw + kKSlots,      // local (x2), e4m3 cache: this CTA's partner V landed
-    kNumBars = kBarVRaw + kKSlots
+    kNumBars = kBarKRaw + kKSlots
 };
 
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
@@ -165,6 +179,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& out_of_ran
 
 struct Params {
     const __nv_bfloat16* q;        // [bs, rows, 576]
+    const uint8_t* kv;             // [num_pages * 64, 576] bf16 or e4m3
     const int32_t* block_table;    // [bs, bt_stride]
     int64_t bt_stride;
     int32_t max_pages;
@@ -283,13 +298,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
-            // bf16: one arrival + the pair's TMA bytes; e4m3: each CTA's widening warp arrives
-            mbar_init(bar(kBarKFull + s), kFp8 ? 2 : 1);
+            // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the page is one piece
+            // and each CTA's widening warp arrives
+            for (int j = 0; j < kKOps; ++j) mbar_init(bar(kBarKFull + kKOps * s + j), kFp8 ? 2 : 1);
             mbar_init(bar(kBarKEmpty + s), 1);
             mbar_init(bar(kBarQKDone + s), 1);
-            mbar_init(bar(kBarVFull + s), kFp8 ? 2 : 1);
+            mbar_init(bar(kBarVFull + s), (kVTma && !kFp8) ? 1 : 8);
             mbar_init(bar(kBarKRaw + s), 1);
-            mbar_init(bar(kBarVRaw + s), 1);
         }
         // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
         mbar_init(bar(kBarQFull), kFp8 ? 8 : 1 + 8);
@@ -348,13 +363,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         }
     };
 
-    if (warp == 0 || warp == 3) {
+    if (warp == 0 || warp == 2 || warp == 3) {
         // ------------------------------------------------------------ K producers
-        // One 72 KB load per tile (this CTA's page, all 576 columns); a thread's TMA loads
-        // start one after another, so two warps take alternate tiles (and slots).
+        // bf16: each tile's page (this CTA's page, all 576 columns) comes in three 24 KB
+        // pieces, piece j by its own warp (0, 2, 3), each completing its own barrier, so the
+        // S MMAs start on the first piece.  e4m3: one 36 KB load per tile, warps 0 / 3 taking
+        // alternate tiles; the loading warp widens the page in place and signals the leader.
+        constexpr bool alternate = kFp8 || kKOps == 1;   // one load per tile: warps 0 / 3 alternate
+        const int piece = alternate ? 0 : (warp == 0 ? 0 : (warp == 2 ? 1 : 2));
         const uint32_t mine = warp == 3 ? 1u : 0u;
         uint32_t g = 0;
-        bool alive = true;
+        bool alive = !(alternate && warp == 2);
         int ub, kb0, kb1;
         while (alive && iter.next(ub, kb0, kb1)) {
             const int n = tiles_of(kb0, kb1);
@@ -363,7 +382,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, warp == 0);
             for (int i = 0; i < n; ++i, ++g) {
                 const int32_t row = pw.row(kb0 + 2 * i + (int)rank);
-                if ((g & 1u) != mine) continue;
+                if (alternate && (g & 1u) != mine) continue;
                 int ok = 1;
                 const int s = (int)(g & 1u);
                 const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
@@ -374,10 +393,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                             mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
                             tma_load_3d(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0);
                         } else {
-                            if (leader) mbar_arrive_expect_tx(bar(kBarKFull + s), 2 * kKSlotBytes);
-                            tma_load_3d_pair(slot, &k_map, map_to_cta(bar(kBarKFull + s), 0), 0, row, 0);
+                            const uint32_t kf = bar(kBarKFull + kKOps * s + piece);
+                            if (leader) mbar_arrive_expect_tx(kf, 2 * kKOpChunks * kBox);
+                            tma_load_3d_pair(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0, row,
+                                             piece * kKOpChunks);
                         }
-                        MLA_TRACE_EVENT(g, 12);
+                        if (piece == 0) MLA_TRACE_EVENT(g, 12);
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
@@ -395,72 +416,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     for (int c = 0; c < kChunks; ++c)
                         widen_chunk_e4m3(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
                     fence_proxy_async_smem();
-                    arrive_leader(kBarKFull + s);
-                }
-            }
-        }
-        if (lane == 0 && *abort_flag) {
-            // let copies already issued land before shared memory can go away
-            const uint64_t t0 = global_timer_ns();
-            while (global_timer_ns() - t0 < 200000ull) {
-            }
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ partner V producer
-        // After a tile's S MMAs, the four chunks of the partner page this CTA supplies to the
-        // PV MMAs (columns 256n + 128r + [0, 128), n = 0, 1) go into the slot positions
-        // 4n + 2(1 - r), + 1, which held this CTA's own, now dead, chunks.
-        uint32_t g = 0;
-        bool alive = true;
-        int ub, kb0, kb1;
-        while (alive && iter.next(ub, kb0, kb1)) {
-            const int n = tiles_of(kb0, kb1);
-            if (n <= 0) continue;
-            PageWindow pw;
-            pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, false);
-            for (int i = 0; i < n; ++i, ++g) {
-                const int32_t row = pw.row(kb0 + 2 * i + 1 - (int)rank);
-                int ok = 1;
-                const int s = (int)(g & 1u);
-                const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
-                if (lane == 0) {
-                    ok = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
-                    if (ok) {
-                        if constexpr (kFp8) {
-                            // e4m3 chunks land in the back half of their 16 KB target region
-                            mbar_arrive_expect_tx(bar(kBarVRaw + s), 2 * 2 * kChunk8);
-#pragma unroll
-                            for (int nn = 0; nn < 2; ++nn)
-                                tma_load_3d(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox + kBox, &v_map,
-                                            bar(kBarVRaw + s), 0, row, 4 * nn + 2 * (int)rank);
-                        } else {
-                            if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * 2 * kVLoadBytes);
-#pragma unroll
-                            for (int nn = 0; nn < 2; ++nn)
-                                tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
-                                                 map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
-                        }
-                        MLA_TRACE_EVENT(g, 18);
-                    }
-                }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) {
-                    alive = false;
-                    break;
-                }
-                if constexpr (kFp8) {
-                    const bool landed = mbar_wait_bounded<false>(bar(kBarVRaw + s), (g >> 1) & 1u, abort_flag);
-                    if (!__all_sync(0xffffffffu, landed)) {
-                        alive = false;
-                        break;
-                    }
-#pragma unroll 1
-                    for (int nn = 0; nn < 2; ++nn) {
-                        const uint32_t region = slot + (4 * nn + 2 * (1 - (int)rank)) * kBox;
-                        widen_chunk_e4m3(region + kBox, region, lane);
-                        widen_chunk_e4m3(region + kBox + kChunk8, region + kBox, lane);
-                    }
-                    fence_proxy_async_smem();
-                    arrive_leader(kBarVFull + s);
+                    arrive_leader(kBarKFull + kKOps * s);
                 }
             }
         }
@@ -471,15 +427,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             }
         }
     } else if (warp >= kQWarp0) {
-        // ------------------------------------------------------------ Q loaders
+        // ------------------------------------------------------------ Q and partner V
         // Per unit, once the previous unit's last S MMA has finished: warp kQWarp0 + 3
-        // (lane 0) loads Q columns [256, 576) of the CTA's 64 rows by TMA, and the four warps
-        // write Q columns [0, 256) into tensor memory, thread = lane.  A pair MMA reads an A
-        // operand from tensor memory for output columns [0, N/2) in lanes 0..63 and for
-        // [N/2, N) in lanes 64..127, so each row lies twice: lane r and lane 64 + r.
+        // (lane 0) loads Q columns [256, 576) of the CTA's 64 rows by TMA (bf16 cache), and
+        // the four warps write Q columns [0, 256) into tensor memory, thread = lane.  A pair
+        // MMA reads an A operand from tensor memory for output columns [0, N/2) in lanes
+        // 0..63 and for [N/2, N) in lanes 64..127, so each row lies twice: lane r and 64 + r.
+        // Per tile, the 128 threads load the four chunks of the partner page this CTA
+        // supplies to the PV MMAs (columns 256n + 128r + [0, 128), n = 0, 1; an L2 hit, the
+        // partner CTA loads that page) into registers ahead of time, and once the tile's S
+        // MMAs are done store them (widened to f16 from an e4m3 cache) into the slot
+        // positions 4n + 2(1 - r), + 1, which held this CTA's own, now dead, chunks.
         // Warp kQWarp0 + 2 (lane 0) first prefetches the query rows of the part's later
         // units into L2.
         const int quarter = warp & 3;
+        const int qt = threadIdx.x - kQWarp0 * 32;          // 0..127
         const int rloc = (32 * quarter + lane) & 63;
         const int rowg = mtile * kRows + kCtaRows * (int)rank + rloc;
         const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
@@ -496,11 +458,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 first = false;
             }
         }
-        uint32_t uq = 0;
-        bool q_range = false;
+        uint32_t uq = 0, g = 0;
+        bool q_range = false, alive = true;
         int ub, kb0, kb1;
-        while (iter.next(ub, kb0, kb1)) {
-            if (tiles_of(kb0, kb1) <= 0) continue;
+        while (alive && iter.next(ub, kb0, kb1)) {
+            const int n = tiles_of(kb0, kb1);
+            if (n <= 0) continue;
+            // ---- Q of the unit
             if (uq > 0 && !mbar_wait_bounded<false>(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
             tc_fence_after();
             if (!kFp8 && quarter == 3 && lane == 0) {
@@ -509,24 +473,26 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                  mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, ub);
             }
             const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)ub * p.rows + rowg) * kDqk);
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                uint4 v[4];
+            {
+                uint4 v[32];   // the row's columns [0, 256): all loads in flight at once
 #pragma unroll
-                for (int k = 0; k < 4; ++k) v[k] = rowg < p.rows ? __ldg(src + 4 * c + k) : make_uint4(0, 0, 0, 0);
-                uint32_t w[16];
+                for (int k = 0; k < 32; ++k) v[k] = rowg < p.rows ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    w[4 * k] = v[k].x;
-                    w[4 * k + 1] = v[k].y;
-                    w[4 * k + 2] = v[k].z;
-                    w[4 * k + 3] = v[k].w;
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        w[4 * k] = v[4 * c + k].x;
+                        w[4 * k + 1] = v[4 * c + k].y;
+                        w[4 * k + 2] = v[4 * c + k].z;
+                        w[4 * k + 3] = v[4 * c + k].w;
+                    }
+                    if constexpr (kFp8) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], q_range);
+                    }
+                    tmem_st16(tmem + lane_off + kTmemQ + 16u * c, w);
                 }
-                if constexpr (kFp8) {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], q_range);
-                }
-                tmem_st16(tmem + lane_off + kTmemQ + 16u * c, w);
             }
             if constexpr (kFp8) {
                 // Q columns [256, 576) as f16 into shared memory (128-byte swizzle): lane
@@ -535,13 +501,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 #pragma unroll 1
                 for (int cc = c0; cc < c1; ++cc) {
                     const uint32_t qrow = sbase + kOffQ + cc * kBox + (uint32_t)rloc * 128u;
+                    uint4 v[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint4 v = rowg < p.rows ? __ldg(src + 32 + 8 * cc + u) : make_uint4(0, 0, 0, 0);
+                    for (int u = 0; u < 8; ++u) v[u] = rowg < p.rows ? __ldg(src + 32 + 8 * cc + u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
                         st_shared_v4u(qrow + 16u * ((uint32_t)u ^ ((uint32_t)rloc & 7u)),
-                                      bf16x2_to_f16x2(v.x, q_range), bf16x2_to_f16x2(v.y, q_range),
-                                      bf16x2_to_f16x2(v.z, q_range), bf16x2_to_f16x2(v.w, q_range));
-                    }
+                                      bf16x2_to_f16x2(v[u].x, q_range), bf16x2_to_f16x2(v[u].y, q_range),
+                                      bf16x2_to_f16x2(v[u].z, q_range), bf16x2_to_f16x2(v[u].w, q_range));
                 }
                 fence_proxy_async_smem();
                 if (__any_sync(0xffffffffu, q_range) && lane == 0) raise_error(32 /* MLA_DEVERR_Q_RANGE */);
@@ -550,9 +517,98 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             tc_fence_before();
             arrive_leader(kBarQFull);
             ++uq;
+            // ---- partner V of each tile of the unit
+            const int32_t* bt_row = p.block_table + (int64_t)ub * p.bt_stride;
+            for (int i = 0; i < n; ++i, ++g) {
+                const int blk = kb0 + 2 * i + 1 - (int)rank;
+                int pg = blk < kb1 ? __ldg(bt_row + blk) : -1;
+                if (pg < 0 || (int64_t)pg >= p.num_pages) pg = -1;   // reported by the K loads
+                const int s = (int)(g & 1u);
+                const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
+                if constexpr (kVTma && !kFp8) {
+                    // by TMA, after the tile's S MMAs: two 16 KB loads, lane 0 of the last warp
+                    if (quarter == 3) {
+                        int ok = 1;
+                        if (lane == 0) {
+                            ok = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                            if (ok) {
+                                if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * 2 * 2 * kBox);
+                                const int32_t row = pg >= 0 ? pg * kPage : (int32_t)(p.num_pages * kPage);
+#pragma unroll
+                                for (int nn = 0; nn < 2; ++nn)
+                                    tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
+                                                     map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
+                                MLA_TRACE_EVENT(g, 18);
+                            }
+                        }
+                        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                            alive = false;
+                            break;
+                        }
+                    }
+                    continue;
+                }
+                if constexpr (kFp8) {
+                    // 4 chunks x 64 rows x 4 sixteen-byte units of e4m3: 8 per thread
+                    uint4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int x = qt + 128 * j, h = x >> 8, row = (x >> 2) & 63, q4 = x & 3;
+                        const int chunk = 4 * (h >> 1) + 2 * (int)rank + (h & 1);
+                        v[j] = pg >= 0 ? __ldg(reinterpret_cast<const uint4*>(
+                                             p.kv + ((int64_t)pg * kPage + row) * kDqk + chunk * 64 + q4 * 16))
+                                       : make_uint4(0, 0, 0, 0);
+                    }
+                    const bool done = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                    if (!__all_sync(0xffffffffu, done)) {
+                        alive = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int x = qt + 128 * j, h = x >> 8, row = (x >> 2) & 63, q4 = x & 3;
+                        const int pos = 4 * (h >> 1) + 2 * (1 - (int)rank) + (h & 1);
+                        const uint32_t r = slot + pos * kBox + row * 128;
+                        const uint32_t sw = (uint32_t)row & 7u;
+                        st_shared_v4u(r + 16u * ((2u * q4) ^ sw), e4m3x2_to_f16x2(v[j].x), e4m3x2_to_f16x2(v[j].x >> 16),
+                                      e4m3x2_to_f16x2(v[j].y), e4m3x2_to_f16x2(v[j].y >> 16));
+                        st_shared_v4u(r + 16u * ((2u * q4 + 1u) ^ sw), e4m3x2_to_f16x2(v[j].z),
+                                      e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w),
+                                      e4m3x2_to_f16x2(v[j].w >> 16));
+                    }
+                } else {
+                    // 4 chunks x 64 rows x 8 sixteen-byte units of bf16: 16 per thread
+                    uint4 v[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int x = qt + 128 * j, h = x >> 9, row = (x >> 3) & 63, u = x & 7;
+                        const int chunk = 4 * (h >> 1) + 2 * (int)rank + (h & 1);
+                        v[j] = pg >= 0 ? __ldg(reinterpret_cast<const uint4*>(
+                                             p.kv + ((int64_t)pg * kPage + row) * (2 * kDqk) + chunk * 128 + u * 16))
+                                       : make_uint4(0, 0, 0, 0);
+                    }
+                    if (qt == 0) MLA_TRACE_EVENT(g, 19);
+                    const bool done = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                    if (!__all_sync(0xffffffffu, done)) {
+                        alive = false;
+                        break;
+                    }
+                    if (qt == 0) MLA_TRACE_EVENT(g, 20);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int x = qt + 128 * j, h = x >> 9, row = (x >> 3) & 63, u = x & 7;
+                        const int pos = 4 * (h >> 1) + 2 * (1 - (int)rank) + (h & 1);
+                        st_shared_v4u(slot + pos * kBox + row * 128 + 16u * ((uint32_t)u ^ ((uint32_t)row & 7u)),
+                                      v[j].x, v[j].y, v[j].z, v[j].w);
+                    }
+                }
+                if (qt == 0) MLA_TRACE_EVENT(g, 18);
+                fence_proxy_async_smem();
+                arrive_leader(kBarVFull + s);
+            }
         }
         if (!kFp8 && quarter == 3 && lane == 0 && *abort_flag) {
-            // let a Q copy already issued land before shared memory can go away
+            // let copies already issued land before shared memory can go away
             const uint64_t t0 = global_timer_ns();
             while (global_timer_ns() - t0 < 200000ull) {
             }
@@ -568,7 +624,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         if (leader && lane == 0) {
             struct Cursor {
                 UnitIter it;
-                int n, i;
+                int n, i, piece;
                 uint32_t g, uq;
                 bool valid;
                 __device__ void next_unit() {
@@ -585,6 +641,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 __device__ void step() {
                     ++g;
+                    piece = 0;
                     if (++i == n) {
                         ++uq;
                         next_unit();
@@ -595,6 +652,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             cq.it = iter;
             cq.g = 0;
             cq.uq = 0;
+            cq.piece = 0;
             cq.next_unit();
             cp = cq;
             uint64_t t_idle = global_timer_ns();
@@ -603,9 +661,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (cp.valid && cp.g < cq.g) {
                     const int s = (int)(cp.g & 1u);
                     const bool first = cp.i == 0;
-                    if (mbar_try_wait_cluster(bar(kBarPFull), cp.g & 1u) &&
-                        mbar_try_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
-                        (!first || cp.uq == 0 || mbar_try_wait_cluster(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
+                    if (mbar_test_wait_cluster(bar(kBarPFull), cp.g & 1u) &&
+                        mbar_test_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
+                        (!first || cp.uq == 0 || mbar_test_wait_cluster(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
                         tc_fence_after();
                         MLA_TRACE_EVENT(cp.g, 2);
                         const uint32_t pbuf = sbase + kOffP;
@@ -628,33 +686,42 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     }
                 }
                 if (!did && cq.valid) {
+                    // S in the pieces the page arrives in (one piece for an e4m3 cache)
                     const int s = (int)(cq.g & 1u);
                     const uint32_t sb = cq.g & 1u;
-                    if ((cq.i != 0 || mbar_try_wait_cluster(bar(kBarQFull), cq.uq & 1u)) &&
-                        (cq.g < 2 || mbar_try_wait_cluster(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
-                        mbar_try_wait_cluster(bar(kBarKFull + s), (cq.g >> 1) & 1u)) {
+                    const int j = cq.piece;
+                    if ((j != 0 || cq.i != 0 || mbar_test_wait_cluster(bar(kBarQFull), cq.uq & 1u)) &&
+                        (j != 0 || cq.g < 2 || mbar_test_wait_cluster(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
+                        mbar_test_wait_cluster(bar(kBarKFull + kKOps * s + (kFp8 ? 0 : j)), (cq.g >> 1) & 1u)) {
                         tc_fence_after();
-                        MLA_TRACE_EVENT(cq.g, 15);
+                        MLA_TRACE_EVENT(cq.g, 15 + j);
                         const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                         const uint32_t d = tmem + kTmemS + 64u * sb;
 #pragma unroll
-                        for (int c = 0; c < kQLoChunks; ++c)
+                        for (int cc = 0; cc < kKOpChunks; ++cc) {
+                            const int c = kKOpChunks * j + cc;
+                            if (c < kQLoChunks) {
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_pair_ts(d, tmem + kTmemQ + 32u * c + 8u * kk,
-                                            smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
-                                            kFp8 ? kIdescQK16 : kIdescQK, (c | kk) ? 1u : 0u);
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_pair_ts(d, tmem + kTmemQ + 32u * c + 8u * kk,
+                                                smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                                kFp8 ? kIdescQK16 : kIdescQK, (c | kk) ? 1u : 0u);
+                            } else {
 #pragma unroll
-                        for (int c = kQLoChunks; c < kChunks; ++c)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_pair_ss(d, smem_desc_sw128(sbase + kOffQ + (c - kQLoChunks) * kBox + 32u * kk, 16, 1024),
-                                            smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
-                                            kFp8 ? kIdescQK16 : kIdescQK, 1u);
-                        tc_commit_pair(bar(kBarQKDone + s));
-                        tc_commit_pair(bar(kBarSFull + sb));
-                        if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
-                        cq.step();
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_pair_ss(d, smem_desc_sw128(sbase + kOffQ + (c - kQLoChunks) * kBox + 32u * kk, 16, 1024),
+                                                smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                                kFp8 ? kIdescQK16 : kIdescQK, 1u);
+                            }
+                        }
+                        if (j == kKOps - 1) {
+                            tc_commit_pair(bar(kBarQKDone + s));
+                            tc_commit_pair(bar(kBarSFull + sb));
+                            if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
+                            cq.step();
+                        } else {
+                            ++cq.piece;
+                        }
                         did = true;
                     }
                 }

@@ -180,9 +180,8 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // Tensor maps (bf16, 128-byte swizzle; coordinates past an extent read as zeros).  Each
     // view orders its dimensions so that one load lands as consecutive 64-row x 64-column
     // boxes (8 KB each), the layout the MMAs read:
-    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = one page, all
-    //      576 columns (72 KB); also the box of the L2 prefetches.
-    //   V: the same view; a load = 2 column chunks of one page (16 KB).
+    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = 3 column
+    //      chunks of one page (24 KB).
     //   Q: (64 columns, rows of a request [1152 B], 9 column chunks [128 B], requests); a load
     //      = 64 query rows x columns [256, 576) (40 KB).
     const int32_t rows = q_len * h_q;
@@ -195,7 +194,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     if (!fp8) {
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {1152, 128};
-        const cuuint32_t kbox[3] = {64, 64, 9};
+        const cuuint32_t kbox[3] = {64, 64, (cuuint32_t)mla::decode::kKOpChunks};
         const cuuint32_t vbox[3] = {64, 64, 2};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), gdim, gstride,
@@ -212,16 +211,12 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {576, 64};
         const cuuint32_t kbox[3] = {64, 64, 9};
-        const cuuint32_t vbox[3] = {64, 64, 2};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(k_cache), gdim, gstride,
                    kbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MLA_ERR_CUDA;
-        if (encode(&v_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(k_cache), gdim, gstride,
-                   vbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return MLA_ERR_CUDA;
+        v_map = k_map;   // the e4m3 path reads partner V through registers
     }
     {
         const cuuint64_t gdim[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)bs};
@@ -237,6 +232,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     const size_t splits = (size_t)bs + (size_t)num_sm_parts;
     mla::decode::Params p;
     p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kv = static_cast<const uint8_t*>(k_cache);
     p.block_table = block_table;
     p.bt_stride = block_table_stride;
     p.max_pages = max_pages;

@@ -74,6 +74,20 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+// Non-blocking tests (never suspend the thread): for a thread that polls several barriers
+// and must react to whichever completes first.
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait budget for one pipeline wait.  Every wait in the kernels is bounded: after this
 // many nanoseconds without the phase completing the waiter records
 // MLA_DEVERR_WAIT_TIMEOUT, raises the CTA's abort flag and returns false; a raised abort
