@@ -84,6 +84,32 @@ def job_value(world, kv_bytes_per_replica, step_ms):
     return world * kv_bytes_per_replica / (step_ms * 1e-3) / 1e9
 
 
+TRAFFIC_KEYS = {2: "deepseek_v3_decode"}
+
+
+def kernel_sources_sha():
+    import hashlib
+    import glob
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_mla_create_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(config):
+    """DRAM bytes per decode launch from the committed ncu capture of this workload, or None
+    when there is none or the kernel sources changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(TRAFFIC_KEYS.get(config, ""), None)
+        if rec and rec["csrc_sha256_prefix"] == kernel_sources_sha():
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -400,7 +426,8 @@ def run_b200(args):
     else:
         roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"]}
-    roof.update({"traffic": None, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
+    roof.update({"traffic": captured_traffic(args.config), "traffic_unit": "bytes per launch",
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
                  if peak_src == "measured" else "fallback",
                  "kernel": "mla_decode_paged call (decode kernel + split merge)",
                  "roofline_time_us": max(t_hbm, t_tc) * 1e6,
