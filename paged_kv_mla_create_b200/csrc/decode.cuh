@@ -88,6 +88,19 @@ constexpr int kKSlotBytes = kChunks * kBox;        // 72 KB: one page, all 576 c
 // warps (S starting on the first piece), and the bf16 partner V through registers like the
 // e4m3 one, were each slower on B200 than one 72 KB load and a TMA load of the partner V
 // (the SM's TMA unit and its global loads share one path; more, smaller requests cost more).
+#ifndef MLA_L2_PREFETCH
+#define MLA_L2_PREFETCH 1
+#endif
+// A K warp that has issued its tile's page load asks the L2, through the load/store path,
+// for the page of its next tile (two tiles on), so that load finds the page in L2.  (A TMA
+// prefetch would queue in the same TMA unit as the loads, which measured slower.)
+constexpr bool kL2Prefetch = MLA_L2_PREFETCH != 0;
+#ifndef MLA_P_SIGNAL_ONCE
+#define MLA_P_SIGNAL_ONCE 0
+#endif
+// The peer CTA's softmax warps signal "P written" to the leader's barrier: each warp with a
+// remote release arrive (0), or once per CTA after a local barrier (1).
+constexpr bool kPSignalOnce = MLA_P_SIGNAL_ONCE != 0;
 constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
 constexpr int kKOpChunks = kChunks / kKOps;
 constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
@@ -128,6 +141,7 @@ enum : int {
     kBarOEmpty,                         // leader: 8 softmax warps read O out
     kBarXchg,                           // local (x2): the 128 softmax threads posted row maxima
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
+    kBarPLocal,                         // local: this CTA's 4 softmax warps wrote P (peer CTA)
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
 };
@@ -296,6 +310,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int part = blockIdx.x >> 1;
     const int mtile = blockIdx.y;
 
+#ifdef MLA_TRACE
+    if (blockIdx.x < 2 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x)
+            (&g_trace[blockIdx.x][0][0])[i] = 0;
+#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
             // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the page is one piece
@@ -313,7 +332,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_init(bar(kBarSFull + j), 1);
             mbar_init(bar(kBarSFree + j), 8);
         }
-        mbar_init(bar(kBarPFull), 8);
+        mbar_init(bar(kBarPFull), kPSignalOnce ? 5 : 8);
+        mbar_init(bar(kBarPLocal), 4);
         mbar_init(bar(kBarPvDone), 1);
         mbar_init(bar(kBarOFull), 1);
         mbar_init(bar(kBarOEmpty), 8);
@@ -404,6 +424,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     alive = false;
                     break;
+                }
+                if constexpr (kL2Prefetch) {
+                    const int blk_next = kb0 + 2 * (i + 2) + (int)rank;
+                    if (alternate && blk_next < kb1) {
+                        const int pn = __ldg(p.block_table + (int64_t)ub * p.bt_stride + blk_next);
+                        if (pn >= 0 && (int64_t)pn < p.num_pages) {
+                            constexpr int kRowBytes = kFp8 ? kDqk : 2 * kDqk;
+                            const uint8_t* base = p.kv + (int64_t)pn * kPage * kRowBytes;
+                            for (int l = lane; l < kPage * kRowBytes / 128; l += 32) prefetch_l2(base + 128 * l);
+                        }
+                    }
                 }
                 if constexpr (kFp8) {
                     // the whole warp widens the page in place, then signals the leader
@@ -661,6 +692,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (cp.valid && cp.g < cq.g) {
                     const int s = (int)(cp.g & 1u);
                     const bool first = cp.i == 0;
+#ifdef MLA_TRACE
+                    if (blockIdx.x < 2 && blockIdx.y == 0 && cp.g < (uint32_t)kTraceTiles) {
+                        if (!g_trace[0][cp.g][21] && mbar_test_wait_cluster(bar(kBarPFull), cp.g & 1u))
+                            g_trace[0][cp.g][21] = clock64();
+                        if (!g_trace[0][cp.g][22] && mbar_test_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u))
+                            g_trace[0][cp.g][22] = clock64();
+                    }
+#endif
                     if (mbar_test_wait_cluster(bar(kBarPFull), cp.g & 1u) &&
                         mbar_test_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
                         (!first || cp.uq == 0 || mbar_test_wait_cluster(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
@@ -877,7 +916,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                       __float_as_uint(s[4 * c + 3]));
                 }
                 fence_proxy_async_smem();
-                arrive_leader(kBarPFull);
+                if (t == 0) MLA_TRACE_EVENT(g, 23);
+                if (kPSignalOnce && !leader) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarPLocal));
+                    if (t == 0) {
+                        if (mbar_wait_bounded<false>(bar(kBarPLocal), g & 1u, abort_flag))
+                            mbar_arrive_remote(map_to_cta(bar(kBarPFull), 0));
+                    }
+                } else {
+                    arrive_leader(kBarPFull);
+                }
                 if (t == 0) MLA_TRACE_EVENT(g, 6);
             }
             if (!alive) break;

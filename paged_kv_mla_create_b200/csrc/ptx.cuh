@@ -168,6 +168,11 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Hint the L2 to fetch the 128-byte line holding addr (no data returns to the SM).
+__device__ __forceinline__ void prefetch_l2(const void* addr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (TMA / tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
