@@ -5,7 +5,7 @@ One step = one pass of the whole path over one batch: page table (build_block_ta
 split plan (get_mla_metadata) and attention with its split merge (mla_decode_paged),
 on inputs resident in HBM.  Default workload: the DeepSeek-V3-shaped decode (bs 64,
 128 heads, q_len 1, L ~ U[1024, 4096], bf16 latent KV 576 wide, 64-token pages in a
-shuffled pool 1.25x the need).  L2 is flushed (a 512 MB write) between timed steps,
+shuffled pool 1.25x the need).  L2 is flushed (512 MB written, then 512 MB read) between timed steps,
 outside the step's CUDA events.
 
 Reported (one JSON line on rank 0):
@@ -140,7 +140,8 @@ def workload_config(cfg_index, wl, world, flush_mb):
     return {"workload": c["name"], "batch": wl.bs, "heads": wl.h, "q_len": wl.q_len,
             "kv_dtype": "fp8_e4m3" if wl.is_fp8 else "bf16", "page": 64,
             "head_dim": 576, "head_dim_v": 512,
-            "l2": f"flushed between timed steps ({flush_mb} MB write, outside the step events)",
+            "l2": f"flushed between timed steps ({flush_mb} MB written, then another {flush_mb} MB read, "
+                  "outside the step events: no input of the step and no dirty line left in L2)",
             "launch": "each step replays CUDA graphs of the metadata and attention calls",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -310,6 +311,11 @@ def run_b200(args):
     lse = torch.empty((bs, q_len, h), dtype=torch.float32, device=dev)
     ws = torch.empty((mla.workspace_bytes(bs, q_len, h, parts),), dtype=torch.uint8, device=dev)
     flush = torch.empty((args.flush_mb << 20,), dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones((args.flush_mb << 20,), dtype=torch.uint8, device=dev)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        flush_rd.max()   # evicts the written lines while still outside the timed region
 
     def metadata(w):
         mla.build_block_table(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
@@ -324,7 +330,7 @@ def run_b200(args):
 
     stream = torch.cuda.current_stream(dev)
     for i in range(args.warmup):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         metadata(wl)
         attention(wl)
     torch.cuda.synchronize(dev)
@@ -346,7 +352,7 @@ def run_b200(args):
     with torch.cuda.graph(g_attn):
         attention(wl)
     for i in range(3):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         g_meta.replay()
         g_attn.replay()
     torch.cuda.synchronize(dev)
@@ -359,7 +365,7 @@ def run_b200(args):
     torch.cuda.synchronize(dev)
     clocks.start()
     for k in range(K):
-        flush.fill_(k & 0xFF)
+        flush_l2(k)
         ev[k][0].record(stream)
         g_meta.replay()
         ev[k][1].record(stream)
@@ -393,7 +399,7 @@ def run_b200(args):
     ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(KE)]
     torch.cuda.synchronize(dev)
     for k in range(KE):
-        flush.fill_(k & 0xFF)
+        flush_l2(k)
         ee[k][0].record(stream)
         dq.copy_(pin_q, non_blocking=True)
         dsl.copy_(pin_sl, non_blocking=True)

@@ -6,7 +6,8 @@
 // One warp per (request, query row).  Requests with a single piece were written
 // directly by the attention kernel and are skipped here, so the launch needs no host
 // knowledge of the plan.  A warp reads its pieces' lse values, then streams the
-// pieces' 512 fp32 columns (16 per lane, as 4 float4) and writes bf16.
+// pieces' 512 fp32 columns (16 per lane, as 4 float4; four pieces' loads in flight at once)
+// and writes bf16.
 #pragma once
 #include "ptx.cuh"
 
@@ -42,18 +43,33 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int i = 0; i < n; ++i) {
-        const float li = part_lse[(int64_t)(s0 + i) * rows + row];
-        const float w = expf(li - lse);
-        const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
+    // pieces four at a time, all of their loads in flight before any is used
+    for (int i0 = 0; i0 < n; i0 += 4) {
+        float4 v[4][4];
+        float w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 v = src[lane + 32 * k];
-            acc[4 * k + 0] += w * v.x;
-            acc[4 * k + 1] += w * v.y;
-            acc[4 * k + 2] += w * v.z;
-            acc[4 * k + 3] += w * v.w;
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            w[j] = 0.f;
+            if (i < n) {
+                w[j] = expf(part_lse[(int64_t)(s0 + i) * rows + row] - lse);
+                const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[j][k] = __ldg(src + lane + 32 * k);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc[4 * k + 0] += w[j] * v[j][k].x;
+                acc[4 * k + 1] += w[j] * v[j][k].y;
+                acc[4 * k + 2] += w[j] * v[j][k].z;
+                acc[4 * k + 3] += w[j] * v[j][k].w;
+            }
     }
     uint2* dst = reinterpret_cast<uint2*>(out + out_row * 512);
 #pragma unroll

@@ -54,12 +54,21 @@ namespace decode {
 #ifdef MLA_TRACE
 constexpr int kTraceTiles = 64, kTraceEvents = 32;
 __device__ long long g_trace[2][kTraceTiles][kTraceEvents];
+__device__ unsigned long long g_ctatrace[1024][16];
+#define MLA_CTA_EVENT(ev)                                                                 \
+    do {                                                                                  \
+        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                             \
+        if (cta_ < 1024 && (ev) < 16) g_ctatrace[cta_][(ev)] = global_timer_ns();         \
+    } while (0)
 #define MLA_TRACE_EVENT(tile, ev)                                                         \
     do {                                                                                  \
         if (blockIdx.x < 2 && blockIdx.y == 0 && (tile) < (uint32_t)kTraceTiles)          \
             g_trace[blockIdx.x][(tile)][(ev)] = clock64();                                \
     } while (0)
 #else
+#define MLA_CTA_EVENT(ev) \
+    do {                  \
+    } while (0)
 #define MLA_TRACE_EVENT(tile, ev) \
     do {                          \
     } while (0)
@@ -123,7 +132,8 @@ constexpr int kOffQ = 0;                            // Q chunks 4..8
 constexpr int kOffK = kOffQ + kQHiBytes;
 constexpr int kOffP = kOffK + kKSlots * kKSlotBytes;
 constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128 floats, row sums 128
-constexpr int kOffBar = kOffX + 3 * 128 * 4;
+constexpr int kOffStage = kOffX + 3 * 128 * 4;      // epilogue staging: 4 warps x 32 rows x 128 B
+constexpr int kOffBar = kOffStage + 4 * 32 * 128;
 
 enum : int {
     kBarKFull = 0,                      // leader (x slots x pieces): both CTAs' piece j landed
@@ -311,6 +321,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int mtile = blockIdx.y;
 
 #ifdef MLA_TRACE
+    if (threadIdx.x == 0) {
+        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;
+        if (cta_ < 1024)
+            for (int e = 0; e < 16; ++e) g_ctatrace[cta_][e] = 0;
+        MLA_CTA_EVENT(0);
+    }
     if (blockIdx.x < 2 && blockIdx.y == 0)
         for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x)
             (&g_trace[blockIdx.x][0][0])[i] = 0;
@@ -734,6 +750,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         mbar_test_wait_cluster(bar(kBarKFull + kKOps * s + (kFp8 ? 0 : j)), (cq.g >> 1) & 1u)) {
                         tc_fence_after();
                         MLA_TRACE_EVENT(cq.g, 15 + j);
+                        if (j == 0 && cq.i == 0 && cq.uq < 6) MLA_CTA_EVENT(3 + 2 * cq.uq);
                         const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                         const uint32_t d = tmem + kTmemS + 64u * sb;
 #pragma unroll
@@ -943,40 +960,71 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             const float inv = l_run > 0.f ? dk / l_run : 0.f;
             const float lse_val = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f
                                               : -INFINITY;
+            // Each warp holds 32 rows; a step moves 128 bytes of each row (32 fp32 partial
+            // columns, or 64 bf16 output columns) from tensor memory through a per-warp staging
+            // area, so that every global store writes whole 128-byte lines (8 lanes per row).
+            {
+                const uint32_t stage = sbase + kOffStage + (uint32_t)(warp - kSoftmaxWarp0) * 4096u;
+                const int row0 = mtile * kRows + kCtaRows * (int)rank + 32 * ((warp - kSoftmaxWarp0) & 1);
+                const int steps = direct ? 4 : 8;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                // TMEM columns [128 + 32c, +32): output columns 256 * (c / 4) + 128 * half + 32 * (c % 4)
-                uint32_t raw[32];
-                tmem_ld16(tmem + lane_off + kTmemO + 32u * c, *reinterpret_cast<uint32_t(*)[16]>(raw));
-                tmem_ld16(tmem + lane_off + kTmemO + 32u * c + 16u,
-                          *reinterpret_cast<uint32_t(*)[16]>(raw + 16));
-                tc_wait_ld();
-                const int col = 256 * (c >> 2) + 128 * half + 32 * (c & 3);
-                if (row_valid) {
+                for (int st = 0; st < steps; ++st) {
+                    uint32_t w[32];
+                    int col;
                     if (direct) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rowg) * kDv + col);
-                        uint32_t w[16];
+                        // 64 columns: TMEM columns [128 + 64 st, +64) = outputs
+                        // 256 (st / 2) + 128 half + 64 (st % 2) + [0, 64)
+                        uint32_t raw[64];
+                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st, *reinterpret_cast<uint32_t(*)[16]>(raw));
+                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(raw + 16));
+                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 32u, *reinterpret_cast<uint32_t(*)[16]>(raw + 32));
+                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 48u, *reinterpret_cast<uint32_t(*)[16]>(raw + 48));
+                        tc_wait_ld();
+                        if (st == steps - 1) {
+                            tc_fence_before();
+                            arrive_leader_done_reading(kBarOEmpty);   // O is free for the next unit
+                        }
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv,
-                                               __uint_as_float(raw[2 * k + 1]) * inv);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        for (int k = 0; k < 32; ++k)
+                            w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv, __uint_as_float(raw[2 * k + 1]) * inv);
+                        col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
                     } else {
-                        float4* dst = reinterpret_cast<float4*>(
-                            p.part_o + ((int64_t)split * p.rows + rowg) * kDv + col);
+                        // 32 columns: TMEM columns [128 + 32 st, +32) = outputs
+                        // 256 (st / 4) + 128 half + 32 (st % 4) + [0, 32)
+                        tmem_ld16(tmem + lane_off + kTmemO + 32u * st, *reinterpret_cast<uint32_t(*)[16]>(w));
+                        tmem_ld16(tmem + lane_off + kTmemO + 32u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(w + 16));
+                        tc_wait_ld();
+                        if (st == steps - 1) {
+                            tc_fence_before();
+                            arrive_leader_done_reading(kBarOEmpty);   // O is free for the next unit
+                        }
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            dst[k] = make_float4(__uint_as_float(raw[4 * k]) * inv,
-                                                 __uint_as_float(raw[4 * k + 1]) * inv,
-                                                 __uint_as_float(raw[4 * k + 2]) * inv,
-                                                 __uint_as_float(raw[4 * k + 3]) * inv);
+                        for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * inv);
+                        col = 256 * (st >> 2) + 128 * half + 32 * (st & 3);
                     }
+                    // this thread's 128 bytes -> staging row `lane` (16-byte unit k at k ^ (lane & 7))
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        st_shared_v4u(stage + (uint32_t)lane * 128u + 16u * ((uint32_t)k ^ ((uint32_t)lane & 7u)),
+                                      w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    __syncwarp();
+                    // 4 rows per store instruction, 8 lanes (128 contiguous bytes) per row
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = 4 * j + (lane >> 3), u = lane & 7;
+                        const int rg = row0 + r;
+                        const uint4 v = ld_shared_v4u(stage + (uint32_t)r * 128u + 16u * ((uint32_t)u ^ ((uint32_t)r & 7u)));
+                        if (rg < p.rows) {
+                            if (direct)
+                                *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
+                            else
+                                *reinterpret_cast<uint4*>(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u) = v;
+                        }
+                    }
+                    __syncwarp();
                 }
             }
-            tc_fence_before();
-            arrive_leader_done_reading(kBarOEmpty);
+            if (t == 0 && uq < 6) MLA_CTA_EVENT(4 + 2 * uq);
             if (row_valid && half == 0) {
                 if (direct)
                     p.lse[(int64_t)ub * p.rows + rowg] = lse_val;
@@ -989,6 +1037,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) MLA_CTA_EVENT(2);
     cluster_sync();
     if (warp == 1) {
         tc_fence_after();

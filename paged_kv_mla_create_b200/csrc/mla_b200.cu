@@ -345,4 +345,8 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_dump(void* host,
     if (bytes > sizeof(mla::decode::g_trace)) bytes = sizeof(mla::decode::g_trace);
     return (int)cudaMemcpyFromSymbol(host, mla::decode::g_trace, bytes);
 }
+extern "C" __attribute__((visibility("default"))) int mla_ctatrace_dump(void* host, size_t bytes) {
+    if (bytes > sizeof(mla::decode::g_ctatrace)) bytes = sizeof(mla::decode::g_ctatrace);
+    return (int)cudaMemcpyFromSymbol(host, mla::decode::g_ctatrace, bytes);
+}
 #endif
