@@ -107,9 +107,16 @@ constexpr bool kL2Prefetch = MLA_L2_PREFETCH != 0;
 #ifndef MLA_P_SIGNAL_ONCE
 #define MLA_P_SIGNAL_ONCE 0
 #endif
+#ifndef MLA_P_SIGNAL_ASYNC
+#define MLA_P_SIGNAL_ASYNC 1
+#endif
 // The peer CTA's softmax warps signal "P written" to the leader's barrier: each warp with a
-// remote release arrive (0), or once per CTA after a local barrier (1).
+// remote release arrive (0), or once per CTA after a local barrier (1); or (async) each warp
+// with a 4-byte st.async into the leader whose complete_tx lands on the barrier, ordered
+// after the warp's P stores by its fence.proxy.async, while the leader's warps arrive with
+// expect_tx (a remote release arrive measured ~1000 cycles before the leader saw it).
 constexpr bool kPSignalOnce = MLA_P_SIGNAL_ONCE != 0;
+constexpr bool kPSignalAsync = MLA_P_SIGNAL_ASYNC != 0 && !kPSignalOnce;
 constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
 constexpr int kKOpChunks = kChunks / kKOps;
 constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
@@ -133,7 +140,8 @@ constexpr int kOffK = kOffQ + kQHiBytes;
 constexpr int kOffP = kOffK + kKSlots * kKSlotBytes;
 constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128 floats, row sums 128
 constexpr int kOffStage = kOffX + 3 * 128 * 4;      // epilogue staging: 4 warps x 32 rows x 128 B
-constexpr int kOffBar = kOffStage + 4 * 32 * 128;
+constexpr int kOffPSig = kOffStage + 4 * 32 * 128;  // leader: landing words of the peer's P signals
+constexpr int kOffBar = kOffPSig + 64;               // (landing words: P 0..3, V 4..7, K 8)
 
 enum : int {
     kBarKFull = 0,                      // leader (x slots x pieces): both CTAs' piece j landed
@@ -335,10 +343,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         for (int s = 0; s < kKSlots; ++s) {
             // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the page is one piece
             // and each CTA's widening warp arrives
-            for (int j = 0; j < kKOps; ++j) mbar_init(bar(kBarKFull + kKOps * s + j), kFp8 ? 2 : 1);
+            // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the leader's widening warp
+            // arrives, the peer's signals by st.async
+            for (int j = 0; j < kKOps; ++j) mbar_init(bar(kBarKFull + kKOps * s + j), 1);
             mbar_init(bar(kBarKEmpty + s), 1);
             mbar_init(bar(kBarQKDone + s), 1);
-            mbar_init(bar(kBarVFull + s), (kVTma && !kFp8) ? 1 : 8);
+            mbar_init(bar(kBarVFull + s), (kVTma && !kFp8) ? 1 : 4);
             mbar_init(bar(kBarKRaw + s), 1);
         }
         // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
@@ -348,7 +358,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_init(bar(kBarSFull + j), 1);
             mbar_init(bar(kBarSFree + j), 8);
         }
-        mbar_init(bar(kBarPFull), kPSignalOnce ? 5 : 8);
+        mbar_init(bar(kBarPFull), kPSignalOnce ? 5 : (kPSignalAsync ? 4 : 8));
         mbar_init(bar(kBarPLocal), 4);
         mbar_init(bar(kBarPvDone), 1);
         mbar_init(bar(kBarOFull), 1);
@@ -389,6 +399,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 mbar_arrive_remote(map_to_cta(bar(b_idx), 0));
         }
     };
+    // A warp publishing shared-memory data (written with st.shared, then fence.proxy.async by
+    // every writing thread) to the leader's MMA: the leader's warp arrives with expect_tx of 4
+    // bytes, the peer's warp sends a 4-byte st.async whose complete_tx lands on the leader's
+    // barrier (word: a landing slot of its own in the leader).  A remote release arrive took
+    // ~1000 cycles longer to reach the leader.
+    auto signal_leader = [&](int b_idx, int word) {
+        __syncwarp();
+        if (lane == 0) {
+            if (leader)
+                mbar_arrive_expect_tx(bar(b_idx), 4);
+            else
+                st_async_b32(map_to_cta(sbase + kOffPSig + 4u * (uint32_t)word, 0), 0u,
+                             map_to_cta(bar(b_idx), 0));
+        }
+    };
     auto arrive_leader_done_reading = [&](int b_idx) {
         __syncwarp();
         if (lane == 0) {
@@ -416,6 +441,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             if (n <= 0) continue;
             PageWindow pw;
             pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, warp == 0);
+            int nx_ub = -1, nx_kb0 = 0, nx_kb1 = 0;   // the next unit with tiles, for the prefetch
+            {
+                UnitIter pk = iter;
+                int a, b0, b1;
+                while (pk.next(a, b0, b1)) {
+                    if (tiles_of(b0, b1) > 0) {
+                        nx_ub = a;
+                        nx_kb0 = b0;
+                        nx_kb1 = b1;
+                        break;
+                    }
+                }
+            }
             for (int i = 0; i < n; ++i, ++g) {
                 const int32_t row = pw.row(kb0 + 2 * i + (int)rank);
                 if (alternate && (g & 1u) != mine) continue;
@@ -442,9 +480,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     break;
                 }
                 if constexpr (kL2Prefetch) {
-                    const int blk_next = kb0 + 2 * (i + 2) + (int)rank;
-                    if (alternate && blk_next < kb1) {
-                        const int pn = __ldg(p.block_table + (int64_t)ub * p.bt_stride + blk_next);
+                    // this warp's next tile: two tiles on, possibly in the part's next unit
+                    int ti = i + 2, tkb0 = kb0, tkb1 = kb1, tub = ub;
+                    if (ti >= n) {
+                        ti -= n;
+                        tkb0 = nx_kb0;
+                        tkb1 = nx_kb1;
+                        tub = nx_ub;
+                    }
+                    const int blk_next = tkb0 + 2 * ti + (int)rank;
+                    if (alternate && tub >= 0 && blk_next < tkb1) {
+                        const int pn = __ldg(p.block_table + (int64_t)tub * p.bt_stride + blk_next);
                         if (pn >= 0 && (int64_t)pn < p.num_pages) {
                             constexpr int kRowBytes = kFp8 ? kDqk : 2 * kDqk;
                             const uint8_t* base = p.kv + (int64_t)pn * kPage * kRowBytes;
@@ -463,7 +509,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     for (int c = 0; c < kChunks; ++c)
                         widen_chunk_e4m3(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
                     fence_proxy_async_smem();
-                    arrive_leader(kBarKFull + kKOps * s);
+                    signal_leader(kBarKFull + kKOps * s, 8);
                 }
             }
         }
@@ -651,7 +697,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 if (qt == 0) MLA_TRACE_EVENT(g, 18);
                 fence_proxy_async_smem();
-                arrive_leader(kBarVFull + s);
+                signal_leader(kBarVFull + s, 4 + quarter);
             }
         }
         if (!kFp8 && quarter == 3 && lane == 0 && *abort_flag) {
@@ -934,7 +980,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 fence_proxy_async_smem();
                 if (t == 0) MLA_TRACE_EVENT(g, 23);
-                if (kPSignalOnce && !leader) {
+                if (kPSignalAsync) {
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (leader)
+                            mbar_arrive_expect_tx(bar(kBarPFull), 4);
+                        else
+                            st_async_b32(map_to_cta(sbase + kOffPSig + 4u * (uint32_t)(warp - kSoftmaxWarp0), 0), g,
+                                         map_to_cta(bar(kBarPFull), 0));
+                    }
+                } else if (kPSignalOnce && !leader) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(kBarPLocal));
                     if (t == 0) {

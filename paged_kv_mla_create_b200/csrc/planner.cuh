@@ -28,6 +28,15 @@ constexpr int kFixedOverhead = 5;        // blocks of cost charged per piece
 constexpr int kPlannerThreads = 256;
 constexpr int kPlannerSmemLens = 2048;   // requests handled by the per-request walk
 
+// a / q for 0 <= a < 2^31, q >= 1: a float estimate (q_inv = 1 / q) corrected to the exact
+// quotient, much shorter on the walk's dependency chain than an integer division.
+__device__ __forceinline__ int div_small(int a, int q, float q_inv) {
+    int m = __float2int_rz((float)a * q_inv);
+    while (m > 0 && m * q > a) --m;
+    while ((m + 1) * q <= a) ++m;
+    return m;
+}
+
 __global__ void __launch_bounds__(kPlannerThreads)
 get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, int32_t parts,
                         int32_t* __restrict__ md, int32_t* __restrict__ num_splits) {
@@ -55,6 +64,7 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
     // Budgets fit in 32 bits for any table a decode step can address (< 2^31 blocks).
     const int P = (int)((total + parts - 1) / parts) + kFixedOverhead;
     const int Q = P - kFixedOverhead;   // >= 1
+    const float qinv = 1.0f / (float)Q;
 
     if (!staged) {
         // part-by-part walk, lengths from global memory
@@ -115,7 +125,7 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
             } else {
                 x0 = r - kFixedOverhead;          // 1 <= x0 < nb
                 const int rem = nb - x0;          // >= 1
-                const int m = (rem - 1) / Q;      // full middle pieces
+                const int m = div_small(rem - 1, Q, qinv);   // full middle pieces
                 const int last = rem - m * Q;     // 1..Q
                 pieces = 2 + m;
                 i += 1 + m;

@@ -145,6 +145,14 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, flo
         : "memory");
 }
 
+// 4-byte asynchronous store into a peer CTA's shared memory, completing 4 bytes of tx on
+// the peer's mbarrier (cluster addresses for both).
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
