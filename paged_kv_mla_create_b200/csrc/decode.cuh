@@ -98,7 +98,7 @@ constexpr int kKSlotBytes = kChunks * kBox;        // 72 KB: one page, all 576 c
 // e4m3 one, were each slower on B200 than one 72 KB load and a TMA load of the partner V
 // (the SM's TMA unit and its global loads share one path; more, smaller requests cost more).
 #ifndef MLA_L2_PREFETCH
-#define MLA_L2_PREFETCH 1
+#define MLA_L2_PREFETCH 0
 #endif
 // A K warp that has issued its tile's page load asks the L2, through the load/store path,
 // for the page of its next tile (two tiles on), so that load finds the page in L2.  (A TMA
@@ -117,6 +117,13 @@ constexpr bool kL2Prefetch = MLA_L2_PREFETCH != 0;
 // expect_tx (a remote release arrive measured ~1000 cycles before the leader saw it).
 constexpr bool kPSignalOnce = MLA_P_SIGNAL_ONCE != 0;
 constexpr bool kPSignalAsync = MLA_P_SIGNAL_ASYNC != 0 && !kPSignalOnce;
+#ifndef MLA_SIGNAL_ALL
+#define MLA_SIGNAL_ALL 1
+#endif
+// Also "Q written" (after the warp's tensor-memory stores completed) and "S / O read" (after
+// its tensor-memory loads completed) from the peer by st.async; the data is already in place
+// (or already read) when the signal is sent, so a 4-byte complete_tx is all the leader needs.
+constexpr bool kSignalAll = MLA_SIGNAL_ALL != 0;
 constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
 constexpr int kKOpChunks = kChunks / kKOps;
 constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
@@ -141,7 +148,8 @@ constexpr int kOffP = kOffK + kKSlots * kKSlotBytes;
 constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128 floats, row sums 128
 constexpr int kOffStage = kOffX + 3 * 128 * 4;      // epilogue staging: 4 warps x 32 rows x 128 B
 constexpr int kOffPSig = kOffStage + 4 * 32 * 128;  // leader: landing words of the peer's P signals
-constexpr int kOffBar = kOffPSig + 64;               // (landing words: P 0..3, V 4..7, K 8)
+constexpr int kOffBar = kOffPSig + 128;   // landing words: P 0..3, V 4..7, K 8, Q 9..12,
+                                            // S read 16..19, O read 20..23
 
 enum : int {
     kBarKFull = 0,                      // leader (x slots x pieces): both CTAs' piece j landed
@@ -352,17 +360,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_init(bar(kBarKRaw + s), 1);
         }
         // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
-        mbar_init(bar(kBarQFull), kFp8 ? 8 : 1 + 8);
+        mbar_init(bar(kBarQFull), (kFp8 ? 0 : 1) + (kSignalAll ? 4 : 8));
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
-            mbar_init(bar(kBarSFree + j), 8);
+            mbar_init(bar(kBarSFree + j), kSignalAll ? 4 : 8);
         }
         mbar_init(bar(kBarPFull), kPSignalOnce ? 5 : (kPSignalAsync ? 4 : 8));
         mbar_init(bar(kBarPLocal), 4);
         mbar_init(bar(kBarPvDone), 1);
         mbar_init(bar(kBarOFull), 1);
-        mbar_init(bar(kBarOEmpty), 8);
+        mbar_init(bar(kBarOEmpty), kSignalAll ? 4 : 8);
         mbar_init(bar(kBarXchg), 128);
         mbar_init(bar(kBarXchg + 1), 128);
         mbar_init(bar(kBarLx), 128);
@@ -608,7 +616,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             }
             tc_wait_st();
             tc_fence_before();
-            arrive_leader(kBarQFull);
+            if (kSignalAll)
+                signal_leader(kBarQFull, 9 + quarter);
+            else
+                arrive_leader(kBarQFull);
             ++uq;
             // ---- partner V of each tile of the unit
             const int32_t* bt_row = p.block_table + (int64_t)ub * p.bt_stride;
@@ -903,7 +914,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 if (t == 0) MLA_TRACE_EVENT(g, 11);
                 tc_fence_before();
-                arrive_leader_done_reading(kBarSFree + sb);
+                if (kSignalAll)
+                    signal_leader(kBarSFree + sb, 16 + (warp - kSoftmaxWarp0));
+                else
+                    arrive_leader_done_reading(kBarSFree + sb);
                 if (t == 0) MLA_TRACE_EVENT(g, 7);
                 // scale to log2 units, mask, this half's maximum
                 const int kbase = (kb0 + 2 * i) * kPage + kPage * half;
@@ -1037,7 +1051,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_wait_ld();
                         if (st == steps - 1) {
                             tc_fence_before();
-                            arrive_leader_done_reading(kBarOEmpty);   // O is free for the next unit
+                            if (kSignalAll)   // O is free for the next unit
+                                signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));
+                            else
+                                arrive_leader_done_reading(kBarOEmpty);
                         }
 #pragma unroll
                         for (int k = 0; k < 32; ++k)
@@ -1051,7 +1068,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_wait_ld();
                         if (st == steps - 1) {
                             tc_fence_before();
-                            arrive_leader_done_reading(kBarOEmpty);   // O is free for the next unit
+                            if (kSignalAll)   // O is free for the next unit
+                                signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));
+                            else
+                                arrive_leader_done_reading(kBarOEmpty);
                         }
 #pragma unroll
                         for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * inv);
