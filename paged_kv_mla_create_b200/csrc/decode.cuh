@@ -124,6 +124,13 @@ constexpr bool kPSignalAsync = MLA_P_SIGNAL_ASYNC != 0 && !kPSignalOnce;
 // its tensor-memory loads completed) from the peer by st.async; the data is already in place
 // (or already read) when the signal is sent, so a 4-byte complete_tx is all the leader needs.
 constexpr bool kSignalAll = MLA_SIGNAL_ALL != 0;
+#ifndef MLA_ISSUER_POLL_CTA
+#define MLA_ISSUER_POLL_CTA 1
+#endif
+// The MMA issuer's barrier tests acquire at CTA scope (1) or cluster scope (0); the data
+// behind a barrier the peer completes is ordered by the peer's fence.proxy.async and the
+// st.async / TMA complete_tx itself, and the CTA-scope test measured ~1% faster.
+constexpr bool kIssuerPollCta = MLA_ISSUER_POLL_CTA != 0;
 constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
 constexpr int kKOpChunks = kChunks / kKOps;
 constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
@@ -443,6 +450,32 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         const uint32_t mine = warp == 3 ? 1u : 0u;
         uint32_t g = 0;
         bool alive = !(alternate && warp == 2);
+#ifdef MLA_TRACE
+        if (alternate && warp == 2 && leader && lane == 0 && blockIdx.x < 2 && blockIdx.y == 0) {
+            // observer: completion time of each traced tile's barriers (leader CTA)
+            uint32_t total = 0;
+            {
+                UnitIter pk = iter;
+                int a, b0, b1;
+                while (pk.next(a, b0, b1)) total += (uint32_t)max(tiles_of(b0, b1), 0);
+            }
+            if (total > (uint32_t)kTraceTiles) total = kTraceTiles;
+            uint32_t gk = 0, gq = 0, gs = 0, gp = 0, gv = 0, gd = 0;
+            const long long t_start = clock64();
+            while (gd < total && clock64() - t_start < 400000000ll && !*abort_flag) {
+                if (gk < total && mbar_test_wait(bar(kBarKFull + kKOps * (gk & 1u)), (gk >> 1) & 1u))
+                    g_trace[0][gk++][24] = clock64();
+                if (gq < total && mbar_test_wait(bar(kBarQKDone + (gq & 1u)), (gq >> 1) & 1u))
+                    g_trace[0][gq++][25] = clock64();
+                if (gs < total && mbar_test_wait(bar(kBarSFull + (gs & 1u)), (gs >> 1) & 1u))
+                    g_trace[0][gs++][26] = clock64();
+                if (gp < total && mbar_test_wait(bar(kBarPFull), gp & 1u)) g_trace[0][gp++][27] = clock64();
+                if (gv < total && mbar_test_wait(bar(kBarVFull + (gv & 1u)), (gv >> 1) & 1u))
+                    g_trace[0][gv++][28] = clock64();
+                if (gd < total && mbar_test_wait(bar(kBarPvDone), gd & 1u)) g_trace[0][gd++][29] = clock64();
+            }
+        }
+#endif
         int ub, kb0, kb1;
         while (alive && iter.next(ub, kb0, kb1)) {
             const int n = tiles_of(kb0, kb1);
@@ -726,6 +759,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // unit, the unit's Q; PV(t) waits for P(t), the partner V of tile t and, first in a
         // unit, the epilogue of the previous unit having read O.
         if (leader && lane == 0) {
+            // non-blocking barrier test for the polling loop
+            auto poll = [](uint32_t b, uint32_t parity) -> bool {
+                return kIssuerPollCta ? mbar_test_wait(b, parity) : mbar_test_wait_cluster(b, parity);
+            };
             struct Cursor {
                 UnitIter it;
                 int n, i, piece;
@@ -760,22 +797,31 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             cq.next_unit();
             cp = cq;
             uint64_t t_idle = global_timer_ns();
+#ifdef MLA_TRACE
+            uint32_t tr_g = 0xffffffffu;
+            bool tr_p = false, tr_v = false;
+#endif
             while (cq.valid || cp.valid) {
                 bool did = false;
                 if (cp.valid && cp.g < cq.g) {
                     const int s = (int)(cp.g & 1u);
                     const bool first = cp.i == 0;
 #ifdef MLA_TRACE
-                    if (blockIdx.x < 2 && blockIdx.y == 0 && cp.g < (uint32_t)kTraceTiles) {
-                        if (!g_trace[0][cp.g][21] && mbar_test_wait_cluster(bar(kBarPFull), cp.g & 1u))
-                            g_trace[0][cp.g][21] = clock64();
-                        if (!g_trace[0][cp.g][22] && mbar_test_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u))
-                            g_trace[0][cp.g][22] = clock64();
+                    if (tr_g != cp.g) {
+                        tr_g = cp.g;
+                        tr_p = tr_v = false;
+                    }
+                    if (!tr_p && poll(bar(kBarPFull), cp.g & 1u)) {
+                        tr_p = true;
+                        MLA_TRACE_EVENT(cp.g, 21);
+                    }
+                    if (!tr_v && poll(bar(kBarVFull + s), (cp.g >> 1) & 1u)) {
+                        tr_v = true;
+                        MLA_TRACE_EVENT(cp.g, 22);
                     }
 #endif
-                    if (mbar_test_wait_cluster(bar(kBarPFull), cp.g & 1u) &&
-                        mbar_test_wait_cluster(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
-                        (!first || cp.uq == 0 || mbar_test_wait_cluster(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
+                    if (poll(bar(kBarPFull), cp.g & 1u) && poll(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
+                        (!first || cp.uq == 0 || poll(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
                         tc_fence_after();
                         MLA_TRACE_EVENT(cp.g, 2);
                         const uint32_t pbuf = sbase + kOffP;
@@ -793,6 +839,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_commit_pair(bar(kBarKEmpty + s));
                         tc_commit_pair(bar(kBarPvDone));
                         if (cp.i == cp.n - 1) tc_commit_pair(bar(kBarOFull));
+                        MLA_TRACE_EVENT(cp.g, 14);
                         cp.step();
                         did = true;
                     }
@@ -802,9 +849,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     const int s = (int)(cq.g & 1u);
                     const uint32_t sb = cq.g & 1u;
                     const int j = cq.piece;
-                    if ((j != 0 || cq.i != 0 || mbar_test_wait_cluster(bar(kBarQFull), cq.uq & 1u)) &&
-                        (j != 0 || cq.g < 2 || mbar_test_wait_cluster(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
-                        mbar_test_wait_cluster(bar(kBarKFull + kKOps * s + (kFp8 ? 0 : j)), (cq.g >> 1) & 1u)) {
+                    if ((j != 0 || cq.i != 0 || poll(bar(kBarQFull), cq.uq & 1u)) &&
+                        (j != 0 || cq.g < 2 || poll(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
+                        poll(bar(kBarKFull + kKOps * s + (kFp8 ? 0 : j)), (cq.g >> 1) & 1u)) {
                         tc_fence_after();
                         MLA_TRACE_EVENT(cq.g, 15 + j);
                         if (j == 0 && cq.i == 0 && cq.uq < 6) MLA_CTA_EVENT(3 + 2 * cq.uq);
@@ -831,6 +878,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                             tc_commit_pair(bar(kBarQKDone + s));
                             tc_commit_pair(bar(kBarSFull + sb));
                             if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
+                            MLA_TRACE_EVENT(cq.g, 13);
                             cq.step();
                         } else {
                             ++cq.piece;
