@@ -7,18 +7,21 @@
 // directly by the attention kernel and are skipped here, so the launch needs no host
 // knowledge of the plan.  A warp reads its pieces' lse values, then streams the
 // pieces' 512 fp32 columns (16 per lane, as 4 float4; four pieces' loads in flight at once)
-// and writes bf16.
+// and writes bf16; the pieces' rows, kept in L2 by the attention kernel's stores, are then
+// dropped from L2 without a write-back (requests of up to kDiscardMaxPieces pieces).
 #pragma once
 #include "ptx.cuh"
 
 namespace mla {
 
 constexpr int kCombineWarps = 8;
+constexpr int kDiscardMaxPieces = 4;   // requests of up to this many pieces drop their rows from L2
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                       const int32_t* __restrict__ num_splits, int32_t rows,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+    const uint64_t read_pol = l2_policy_evict_first();   // the partials are read once
     const int b = blockIdx.y;
     const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -40,6 +43,10 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
     for (int i = lane; i < n; i += 32) sum += expf(part_lse[(int64_t)(s0 + i) * rows + row] - m);
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     const float lse = m + logf(sum);
+    // A request of few pieces drops its rows' L2 lines once merged (they need no write-back);
+    // the loads of a many-piece request (a long serial loop here) only lower their L2
+    // priority, which measured faster than dropping each line.
+    const bool discard = MLA_L2_HINTS && n <= kDiscardMaxPieces;
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
@@ -55,7 +62,9 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
                 w[j] = expf(part_lse[(int64_t)(s0 + i) * rows + row] - lse);
                 const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) v[j][k] = __ldg(src + lane + 32 * k);
+                for (int k = 0; k < 4; ++k)
+                    v[j][k] = (MLA_L2_HINTS && !discard) ? ld_global_nc_v4_hint(src + lane + 32 * k, read_pol)
+                                                         : __ldg(src + lane + 32 * k);
             } else {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) v[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -70,6 +79,15 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
                 acc[4 * k + 2] += w[j] * v[j][k].z;
                 acc[4 * k + 3] += w[j] * v[j][k].w;
             }
+        if (discard) {
+            // every lane's loads have returned (consumed above): the pieces' rows are dead, so
+            // their L2 lines go without a write-back (lane l < 16 takes line l of a 2 KB row)
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (i0 + j < n && lane < 16)
+                    discard_l2_line(part_o + ((int64_t)(s0 + i0 + j) * rows + row) * 512 + 32 * lane);
+        }
     }
     uint2* dst = reinterpret_cast<uint2*>(out + out_row * 512);
 #pragma unroll

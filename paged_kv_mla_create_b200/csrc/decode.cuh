@@ -135,6 +135,12 @@ constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 
 constexpr int kKOpChunks = kChunks / kKOps;
 constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
 static_assert(kKOps == 1 || kKOps == 3, "page pieces");
+// KV page loads evict-first and split partials evict-last in L2, so that the partials are still
+// in L2 when the merge reads them (the merge then drops their lines without a write-back).
+constexpr bool kL2Hints = MLA_L2_HINTS != 0;
+#ifndef MLA_KV_EVICT_FIRST
+#define MLA_KV_EVICT_FIRST 1
+#endif
 constexpr int kPBytes = 2 * kBox;          // P: 64 rows x 128 tokens bf16
 constexpr int kThreads = 384;              // 12 warps (roles above)
 constexpr int kSoftmaxWarp0 = 4;
@@ -401,6 +407,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     bool md_ok = true;
     UnitIter iter = make_iter(p, part, md_ok);
+    const uint64_t kv_pol = MLA_KV_EVICT_FIRST ? l2_policy_evict_first() : l2_policy_evict_normal();
+    const uint64_t part_pol = l2_policy_evict_last();
     if (!md_ok && threadIdx.x == 0) raise_error(8 /* MLA_DEVERR_BAD_METADATA */);
 
     // Signals to the leader's barriers: the leader's own warps arrive locally; the peer's
@@ -506,12 +514,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     if (ok) {
                         if constexpr (kFp8) {
                             mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
-                            tma_load_3d(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0);
+                            if (kL2Hints)
+                                tma_load_3d_hint(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0, kv_pol);
+                            else
+                                tma_load_3d(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0);
                         } else {
                             const uint32_t kf = bar(kBarKFull + kKOps * s + piece);
                             if (leader) mbar_arrive_expect_tx(kf, 2 * kKOpChunks * kBox);
-                            tma_load_3d_pair(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0, row,
-                                             piece * kKOpChunks);
+                            if (kL2Hints)
+                                tma_load_3d_pair_hint(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0,
+                                                      row, piece * kKOpChunks, kv_pol);
+                            else
+                                tma_load_3d_pair(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0, row,
+                                                 piece * kKOpChunks);
                         }
                         if (piece == 0) MLA_TRACE_EVENT(g, 12);
                     }
@@ -673,8 +688,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                 const int32_t row = pg >= 0 ? pg * kPage : (int32_t)(p.num_pages * kPage);
 #pragma unroll
                                 for (int nn = 0; nn < 2; ++nn)
-                                    tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
-                                                     map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
+                                    if (kL2Hints)
+                                        tma_load_3d_pair_hint(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
+                                                              map_to_cta(bar(kBarVFull + s), 0), 0, row,
+                                                              4 * nn + 2 * (int)rank, kv_pol);
+                                    else
+                                        tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
+                                                         map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
                                 MLA_TRACE_EVENT(g, 18);
                             }
                         }
@@ -1140,6 +1160,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         if (rg < p.rows) {
                             if (direct)
                                 *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
+                            else if (kL2Hints)
+                                st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
                             else
                                 *reinterpret_cast<uint4*>(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u) = v;
                         }
@@ -1151,6 +1173,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             if (row_valid && half == 0) {
                 if (direct)
                     p.lse[(int64_t)ub * p.rows + rowg] = lse_val;
+                else if (kL2Hints)
+                    st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
                 else
                     p.part_lse[(int64_t)split * p.rows + rowg] = lse_val;
             }
