@@ -87,12 +87,16 @@ def job_value(world, kv_bytes_per_replica, step_ms):
 TRAFFIC_KEYS = {2: "deepseek_v3_decode"}
 
 
+# The sources the decode kernel is built from: its body, the PTX helpers it inlines, and the
+# translation unit with its tensor maps and launch configuration.
+DECODE_KERNEL_SOURCES = ("decode.cuh", "ptx.cuh", "mla_b200.cu")
+
+
 def kernel_sources_sha():
     import hashlib
-    import glob
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_mla_create_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for name in DECODE_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_mla_create_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 

@@ -32,6 +32,9 @@ constexpr int kPlannerSmemLens = 2048;   // requests handled by the per-request 
 // quotient, much shorter on the walk's dependency chain than an integer division.
 __device__ __forceinline__ int div_small(int a, int q, float q_inv) {
     int m = __float2int_rz((float)a * q_inv);
+    // one step each way covers the estimate's error for a < 2^22; the loops finish the rest
+    m = (m > 0 && m * q > a) ? m - 1 : m;
+    m = ((m + 1) * q <= a) ? m + 1 : m;
     while (m > 0 && m * q > a) --m;
     while ((m + 1) * q <= a) ++m;
     return m;
@@ -107,33 +110,27 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
     }
 
     if (threadIdx.x == 0) {
+        // Straight-line step: both outcomes (the request fits / it is split) are computed and
+        // one is selected, so an iteration is one short dependency chain through r and i.
         int i = 0, r = P, cum = 0;
         int nb = s_nb[0];
         for (int b = 0; b < bs; ++b) {
             const int nb_next = s_nb[b + 1];
             const int c = nb + kFixedOverhead;
-            if (r < c && r <= kFixedOverhead) {   // the part ends with budget unused
-                ++i;
-                r = P;
-            }
-            int pieces, x0;
+            const bool skip = (r < c) & (r <= kFixedOverhead);   // the part ends with budget unused
+            r = skip ? P : r;
+            i += skip ? 1 : 0;
+            const bool fits = r >= c;
+            const int x0s = r - kFixedOverhead;                   // split: 1 <= x0s < nb
+            const int rem = nb - x0s;                             // split: >= 1
+            const int m = div_small(max(rem - 1, 0), Q, qinv);    // split: full middle pieces
+            const int last = rem - m * Q;                         // split: 1..Q
             s_fp[b] = i;
-            if (r >= c) {
-                pieces = 1;
-                x0 = nb;
-                r -= c;
-            } else {
-                x0 = r - kFixedOverhead;          // 1 <= x0 < nb
-                const int rem = nb - x0;          // >= 1
-                const int m = div_small(rem - 1, Q, qinv);   // full middle pieces
-                const int last = rem - m * Q;     // 1..Q
-                pieces = 2 + m;
-                i += 1 + m;
-                r = P - last - kFixedOverhead;
-            }
+            i = fits ? i : i + 1 + m;
+            r = fits ? r - c : P - last - kFixedOverhead;
             s_lp[b] = i;
-            s_x0[b] = x0;
-            cum += pieces;
+            s_x0[b] = fits ? nb : x0s;
+            cum += fits ? 1 : 2 + m;
             s_cum[b] = cum;
             nb = nb_next;
         }

@@ -205,3 +205,22 @@ def test_full_size_workload_sampled(mla, index):
     # log of one allowed key's weight (lse > -inf) for every live row
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     assert mla.read_device_error() == 0
+
+
+# ------------------------------------------------------------------ planner, random batches
+def test_planner_random_batches(mla):
+    """The device split planner against the oracle's walk, bit-exact, on random batches:
+    zero-length requests, single-block requests and long ones, 1 to 2500 requests (both the
+    per-request walk and the part-by-part walk of batches above 2048), 1 to 148 parts."""
+    rng = np.random.default_rng(20261202)
+    for t in range(300):
+        bs = int(rng.integers(1, 2500 if t % 25 == 0 else 300))
+        kind = rng.integers(0, 4, size=bs)
+        lens = np.where(kind == 0, 0, np.where(kind == 1, rng.integers(1, 65, size=bs),
+                        np.where(kind == 2, rng.integers(1, 8193, size=bs), rng.integers(1, 131073, size=bs))))
+        seqlens = torch.tensor(lens, dtype=torch.int32)
+        parts = int(rng.integers(1, 149))
+        md, ns = mla.get_mla_metadata(seqlens.cuda(), 128, num_parts=parts)
+        ref_md, ref_ns = oracle.get_mla_metadata(seqlens.numpy(), parts)
+        assert np.array_equal(md.cpu().numpy(), ref_md), f"batch {t}: metadata differs (bs {bs}, parts {parts})"
+        assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits differs (bs {bs}, parts {parts})"
