@@ -362,8 +362,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 #endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
-            // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the page is one piece
-            // and each CTA's widening warp arrives
             // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the leader's widening warp
             // arrives, the peer's signals by st.async
             for (int j = 0; j < kKOps; ++j) mbar_init(bar(kBarKFull + kKOps * s + j), 1);
@@ -449,10 +447,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     if (warp == 0 || warp == 2 || warp == 3) {
         // ------------------------------------------------------------ K producers
-        // bf16: each tile's page (this CTA's page, all 576 columns) comes in three 24 KB
-        // pieces, piece j by its own warp (0, 2, 3), each completing its own barrier, so the
-        // S MMAs start on the first piece.  e4m3: one 36 KB load per tile, warps 0 / 3 taking
-        // alternate tiles; the loading warp widens the page in place and signals the leader.
+        // Each tile's page (this CTA's page, all 576 columns) is one load, warps 0 / 3 taking
+        // alternate tiles: 72 KB of bf16 completing the leader's barrier, or 36 KB of e4m3 that
+        // the loading warp widens in place before it signals the leader.  (Built with
+        // MLA_KOPS=3, the bf16 page comes in three 24 KB pieces by warps 0, 2 and 3, each on its
+        // own barrier, so that the S MMAs start on the first piece.)
         constexpr bool alternate = kFp8 || kKOps == 1;   // one load per tile: warps 0 / 3 alternate
         const int piece = alternate ? 0 : (warp == 0 ? 0 : (warp == 2 ? 1 : 2));
         const uint32_t mine = warp == 3 ? 1u : 0u;
@@ -865,7 +864,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     }
                 }
                 if (!did && cq.valid) {
-                    // S in the pieces the page arrives in (one piece for an e4m3 cache)
+                    // S in the pieces the page arrives in (one, unless built with MLA_KOPS=3)
                     const int s = (int)(cq.g & 1u);
                     const uint32_t sb = cq.g & 1u;
                     const int j = cq.piece;

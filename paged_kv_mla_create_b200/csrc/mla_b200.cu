@@ -180,8 +180,9 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // Tensor maps (bf16, 128-byte swizzle; coordinates past an extent read as zeros).  Each
     // view orders its dimensions so that one load lands as consecutive 64-row x 64-column
     // boxes (8 KB each), the layout the MMAs read:
-    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = 3 column
-    //      chunks of one page (24 KB).
+    //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = all nine
+    //      column chunks of one page (72 KB; three chunks, 24 KB, when built with MLA_KOPS=3).
+    //   V: the same view with a box of two column chunks (16 KB): a partner page's V chunks.
     //   Q: (64 columns, rows of a request [1152 B], 9 column chunks [128 B], requests); a load
     //      = 64 query rows x columns [256, 576) (40 KB).
     const int32_t rows = q_len * h_q;
