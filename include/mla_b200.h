@@ -193,7 +193,9 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *   out               bf16 [bs, q_len, h_q, 512] (written)
  *   lse               fp32 [bs, q_len, h_q] natural-log log-sum-exp (written)
  *   workspace         at least mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts)
- *                     bytes, 256-byte aligned; its contents need no initialisation
+ *                     bytes, 256-byte aligned; its contents need no initialisation and are
+ *                     undefined after the call (the merge may drop the split partials'
+ *                     L2 lines without writing them back)
  * Calls on the same workspace that overlap on the GPU race; use one workspace per stream.
  * The first call on a device also sets the kernel's shared-memory limit (a host-side
  * attribute; no allocation).
