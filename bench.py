@@ -114,6 +114,35 @@ def captured_traffic(config):
     return None
 
 
+def roofline_entry(kv_bytes, q_bytes, flops, attn_s, peaks, peak_src, is_fp8, traffic):
+    """The bench line's roofline object for one attention call of attn_s seconds: bound by HBM
+    (algorithmic KV + Q bytes) or by the tensor cores (algorithmic FLOPs at the measured bf16
+    peak; the e4m3 cache computes with f16 MMAs, whose peak is the bf16 one).  An e4m3 cache is
+    also reported against the fp8 peak (the measured bf16 peak x the nominal fp8 / bf16 ratio 2),
+    the rate a path with fp8 MMAs would have."""
+    t_hbm = (kv_bytes + q_bytes) / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    achieved_gbs = (kv_bytes + q_bytes) / attn_s / 1e9
+    achieved_tf = flops / attn_s / 1e12
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"]}
+    roof.update({"traffic": traffic, "traffic_unit": "bytes per launch",
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
+                 if peak_src == "measured" else "fallback",
+                 "kernel": "mla_decode_paged call (decode kernel + split merge)",
+                 "roofline_time_us": max(t_hbm, t_tc) * 1e6,
+                 "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s})
+    if is_fp8:
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        roof.update({"fp8_peak_tflops": fp8_peak, "frac_of_fp8_peak": achieved_tf / fp8_peak,
+                     "fp8_peak_source": "measured bf16 peak x 2 (nominal fp8 / bf16 ratio)"})
+    return roof
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -432,24 +461,10 @@ def run_b200(args):
         raise RuntimeError(f"device error word {int(err)} after the timed run")
 
     peaks, peak_src = load_peaks()
-    t_hbm = (kv_bytes + q_bytes) / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
     attn_s = attn_ms * 1e-3
-    achieved_gbs = (kv_bytes + q_bytes) / attn_s / 1e9
     achieved_tf = flops / attn_s / 1e12
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"]}
-    else:
-        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"]}
-    roof.update({"traffic": captured_traffic(args.config), "traffic_unit": "bytes per launch",
-                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
-                 if peak_src == "measured" else "fallback",
-                 "kernel": "mla_decode_paged call (decode kernel + split merge)",
-                 "roofline_time_us": max(t_hbm, t_tc) * 1e6,
-                 "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s})
+    roof = roofline_entry(kv_bytes, q_bytes, flops, attn_s, peaks, peak_src, host.is_fp8,
+                          captured_traffic(args.config))
 
     if rank != 0:
         if world > 1:
@@ -459,7 +474,8 @@ def run_b200(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if host.is_fp8 else "bf16",
+        "data": "synthetic",
         "config": workload_config(args.config, host, world, args.flush_mb),
         "us_per_call": attn_ms * 1e3, "metadata_us": meta_ms * 1e3,
         "kv_gbs_per_call": kv_bytes / attn_s / 1e9, "tflops": achieved_tf,

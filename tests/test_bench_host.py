@@ -1,0 +1,40 @@
+"""Host-side arithmetic of bench.py's JSON line (no GPU): the roofline object."""
+import json
+import math
+
+import bench
+
+PEAKS = {"hbm_gbs": 6549.4, "bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0}
+
+
+def test_roofline_hbm_bound_decode():
+    # DeepSeek-V3-shaped decode: 198.2 MB of KV + Q, 45.6 GFLOP, one call of 86.9 us
+    kv, q, fl, t = 188.8e6, 9.4e6, 45.6e9, 86.9e-6
+    r = bench.roofline_entry(kv, q, fl, t, PEAKS, "measured", False, 199744256.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert math.isclose(r["achieved"], (kv + q) / t / 1e9)
+    assert math.isclose(r["frac"], r["achieved"] / PEAKS["hbm_gbs"])
+    assert math.isclose(r["roofline_time_us"], (kv + q) / (PEAKS["hbm_gbs"] * 1e9) * 1e6)
+    assert math.isclose(r["frac_of_roofline_time"], r["frac"])   # HBM-bound: the two agree
+    assert r["traffic"] == 199744256.0
+    assert "frac_of_fp8_peak" not in r
+    json.dumps(r)
+
+
+def test_roofline_fp8_cache_reports_both_peaks():
+    # e4m3 cache: half the KV bytes, the same FLOPs -> tensor-bound at the bf16 (f16 MMA) peak,
+    # also reported against the fp8 peak (2x)
+    kv, q, fl, t = 150e6, 18.9e6, 146e9, 256.6e-6
+    r = bench.roofline_entry(kv, q, fl, t, PEAKS, "measured", True, None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert math.isclose(r["achieved"], fl / t / 1e12)
+    assert math.isclose(r["frac"], r["achieved"] / PEAKS["bf16_tflops"])
+    assert math.isclose(r["fp8_peak_tflops"], 2 * PEAKS["bf16_tflops"])
+    assert math.isclose(r["frac_of_fp8_peak"], r["frac"] / 2)
+    assert r["traffic"] is None
+    json.dumps(r)
+
+
+def test_roofline_fallback_peak_is_named():
+    r = bench.roofline_entry(1e9, 0.0, 1e9, 1e-3, bench.FALLBACK_PEAKS, "fallback", False, None)
+    assert r["peak_source"] == "fallback"
