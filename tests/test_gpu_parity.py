@@ -224,3 +224,28 @@ def test_planner_random_batches(mla):
         ref_md, ref_ns = oracle.get_mla_metadata(seqlens.numpy(), parts)
         assert np.array_equal(md.cpu().numpy(), ref_md), f"batch {t}: metadata differs (bs {bs}, parts {parts})"
         assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits differs (bs {bs}, parts {parts})"
+
+
+# ------------------------------------------------------------------ repeated calls, one workspace
+def test_repeated_calls_on_one_workspace_are_identical(mla):
+    """The path has no atomics and a fixed split order, so repeated calls must agree bit for
+    bit; reusing one workspace also checks that a call never depends on what a previous call
+    left in it (the merge drops the partials' L2 lines without writing them back)."""
+    wl = W.make_case([700, 1500, 64, 2300, 1], 128, seed=77)
+    g = wl.to("cuda")
+    bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages)
+    parts = 9   # forces several pieces per request
+    md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, num_parts=parts)
+    ws = torch.empty((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), dtype=torch.uint8, device="cuda")
+    outs = []
+    for k in range(3):
+        if k == 2:
+            ws.fill_(0xFF)   # a workspace full of NaN patterns must not matter either
+        o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                                      wl.causal, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((o.clone(), lse.clone()))
+    for o, lse in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1]), "repeated calls differ"
+    assert int(ns[-1]) > wl.bs, "the case should split requests"
+    assert mla.read_device_error() == 0
