@@ -59,7 +59,7 @@ def _load():
     lib.oracle_num_sm_parts.restype = I64
     lib.oracle_get_mla_metadata.argtypes = [P, I64, I64, I64, P, P]
     lib.oracle_get_mla_metadata.restype = None
-    lib.oracle_mla_decode_rows.argtypes = [P, P, I32, D, D, P, I64, P, P, P, P, I64, I64, I64,
+    lib.oracle_mla_decode_rows.argtypes = [P, I32, P, I32, D, D, P, I64, P, P, P, P, I64, I64, I64,
                                            I64, I64, D, I32, I64, P, P, P]
     lib.oracle_mla_decode_rows.restype = I32
     lib.oracle_merge_states.argtypes = [I64, I64, P, P, P, P]
@@ -133,14 +133,15 @@ def get_mla_metadata(cache_seqlens, num_parts: int,
 def mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, row_ids,
                     softmax_scale: float, causal: bool, head_dim_v: int = 512,
                     kv_is_fp8: bool = False, descale_q: float = 1.0, descale_k: float = 1.0,
-                    key_begin=None, key_end=None):
+                    key_begin=None, key_end=None, q_is_fp8: bool = False):
     """Attention for the flat rows (b * q_len + i) * h + head of q [bs, q_len, h, dq].
 
     kv_cache is the token-slot pool (any shape whose last dim is dq; bf16 or e4m3
-    torch tensors, or their raw uint16 / uint8 bits).  Returns (o [n, dv] fp64,
-    lse [n] fp64).
+    torch tensors, or their raw uint16 / uint8 bits); q is bf16, or e4m3 codes with
+    q_is_fp8 (descale_q then being the scale q was quantised with).  Returns
+    (o [n, dv] fp64, lse [n] fp64).
     """
-    qb = _np(q, np.uint16)
+    qb = _np(q, np.uint8 if q_is_fp8 else np.uint16)
     bs, q_len, h, dq = qb.shape
     kv = _np(kv_cache, np.uint8 if kv_is_fp8 else np.uint16).reshape(-1, dq)
     r2t = _np(req_to_token, np.int32)
@@ -153,7 +154,7 @@ def mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, 
     o = np.empty((n, head_dim_v), dtype=np.float64)
     lse = np.empty((n,), dtype=np.float64)
     rc = _load().oracle_mla_decode_rows(
-        _ptr(qb), _ptr(kv), int(kv_is_fp8), float(descale_q), float(descale_k), _ptr(r2t),
+        _ptr(qb), int(q_is_fp8), _ptr(kv), int(kv_is_fp8), float(descale_q), float(descale_k), _ptr(r2t),
         r2t.shape[1], _ptr(rpi), _ptr(sl), _ptr(kb) if kb is not None else None,
         _ptr(ke) if ke is not None else None, bs, q_len, h, dq, head_dim_v, float(softmax_scale),
         int(causal), n, _ptr(rows), _ptr(o), _ptr(lse))
@@ -164,13 +165,14 @@ def mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, 
 
 def mla_decode(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, softmax_scale: float,
                causal: bool, head_dim_v: int = 512, kv_is_fp8: bool = False,
-               descale_q: float = 1.0, descale_k: float = 1.0, key_begin=None, key_end=None):
+               descale_q: float = 1.0, descale_k: float = 1.0, key_begin=None, key_end=None,
+               q_is_fp8: bool = False):
     """All rows: (o [bs, q_len, h, dv] fp64, lse [bs, q_len, h] fp64)."""
     bs, q_len, h, _ = tuple(q.shape)
     rows = np.arange(bs * q_len * h, dtype=np.int64)
     o, lse = mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, rows,
                              softmax_scale, causal, head_dim_v, kv_is_fp8, descale_q, descale_k,
-                             key_begin, key_end)
+                             key_begin, key_end, q_is_fp8)
     return o.reshape(bs, q_len, h, head_dim_v), lse.reshape(bs, q_len, h)
 
 

@@ -168,12 +168,14 @@ void oracle_get_mla_metadata(const int32_t* cache_seqlens, int64_t bs, int64_t n
  *   o   = sum_j exp(s_j - lse) * v_j
  * With no allowed key: o = 0 and lse = -inf.
  */
-static void attend_row(const uint16_t* q_row, const uint8_t* kv, int kv_is_fp8, double descale_q,
-                       double descale_k, const int32_t* r2t_row, int64_t j_begin, int64_t j_end,
-                       int64_t dq, int64_t dv, double softmax_scale, double* o, double* lse,
-                       double* s_buf) {
+static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int kv_is_fp8,
+                       double descale_q, double descale_k, const int32_t* r2t_row, int64_t j_begin,
+                       int64_t j_end, int64_t dq, int64_t dv, double softmax_scale, double* o,
+                       double* lse, double* s_buf) {
     double qd[1024];
-    for (int64_t d = 0; d < dq; ++d) qd[d] = bf16_bits_to_double(q_row[d]);
+    for (int64_t d = 0; d < dq; ++d)
+        qd[d] = q_is_fp8 ? e4m3_bits_to_double(((const uint8_t*)q_row)[d])
+                         : bf16_bits_to_double(((const uint16_t*)q_row)[d]);
     int64_t n = j_end - j_begin;
     if (n <= 0) {
         for (int64_t d = 0; d < dv; ++d) o[d] = 0.0;
@@ -214,9 +216,12 @@ static void attend_row(const uint16_t* q_row, const uint8_t* kv, int kv_is_fp8, 
  * key_begin / key_end (nullable, indexed by b) restrict request b's keys to a range
  * before the causal limit is applied; null means the whole [0, L).
  * kv is the flat token-slot pool [num_slots, dq] of bf16 bits (kv_is_fp8 = 0) or
- * e4m3 bytes (kv_is_fp8 = 1).  Returns 0, or -1 when the query width exceeds 1024.
+ * e4m3 bytes (kv_is_fp8 = 1); q is [bs, q_len, h, dq] of bf16 bits (q_is_fp8 = 0) or e4m3
+ * bytes (q_is_fp8 = 1: the flash_mla_with_kvcache call of the FlashMLA backend page, with q
+ * quantised by scaled_fp8_quant and descale_q its scale).  Returns 0, or -1 when the query
+ * width exceeds 1024.
  */
-int oracle_mla_decode_rows(const uint16_t* q, const void* kv, int kv_is_fp8, double descale_q,
+int oracle_mla_decode_rows(const void* q, int q_is_fp8, const void* kv, int kv_is_fp8, double descale_q,
                            double descale_k, const int32_t* req_to_token, int64_t r2t_stride,
                            const int64_t* req_pool_indices, const int32_t* cache_seqlens,
                            const int64_t* key_begin, const int64_t* key_end, int64_t bs,
@@ -245,7 +250,9 @@ int oracle_mla_decode_rows(const uint16_t* q, const void* kv, int kv_is_fp8, dou
             int64_t j1 = key_end ? key_end[b] : L;
             if (j0 < 0) j0 = 0;
             if (j1 > lim) j1 = lim;
-            attend_row(q + flat * dq, (const uint8_t*)kv, kv_is_fp8, descale_q, descale_k,
+            const void* q_row = q_is_fp8 ? (const void*)((const uint8_t*)q + flat * dq)
+                                         : (const void*)((const uint16_t*)q + flat * dq);
+            attend_row(q_row, q_is_fp8, (const uint8_t*)kv, kv_is_fp8, descale_q, descale_k,
                        req_to_token + req_pool_indices[b] * r2t_stride, j0, j1, dq, dv,
                        softmax_scale, o_out + r * dv, lse_out + r, s_buf);
         }

@@ -28,6 +28,8 @@ MUTANTS = {
                         "double l = log(sum);\n    for (int64_t d = 0; d < dv; ++d) o[d] = 0.0;"),
     "merge_weight_uses_max": ("double w = exp(lse_parts[k] - l);",
                               "double w = exp(lse_parts[k] - m);"),
+    "fp8_query_neighbours_swapped": ("qd[d] = q_is_fp8 ? e4m3_bits_to_double(((const uint8_t*)q_row)[d])",
+                                     "qd[d] = q_is_fp8 ? e4m3_bits_to_double(((const uint8_t*)q_row)[d ^ 1])"),
     "descale_k_dropped": ("? e4m3_bits_to_double(kv[slot * dq + d]) * descale_k\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc",
                           "? e4m3_bits_to_double(kv[slot * dq + d])\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc"),
 }

@@ -388,6 +388,30 @@ def test_fp8_equals_bf16_on_dequantized_cache():
     assert np.array_equal(o8, ob) and np.array_equal(l8, lb)
 
 
+def test_fp8_query_equals_bf16_query_on_its_values():
+    """A query given as e4m3 codes (the FlashMLA backend page quantises q with
+    scaled_fp8_quant before the call, descale_q being the scale): every e4m3 value is exact in
+    bf16, so the oracle on the codes must equal the oracle on a bf16 q holding their values,
+    with the same descale_q, on a bf16 and on an e4m3 cache."""
+    for kv in ("bf16", "fp8"):
+        wl = W.make_case([90, 200, 1], h=4, kv=kv, seed=18)
+        scale = 0.03125
+        codes = (wl.q.to(torch.float32) / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+        vals = codes.to(torch.bfloat16)
+        assert torch.equal(vals.to(torch.float64), codes.to(torch.float64))
+        dk = float(wl.descale_k[0]) if wl.descale_k is not None else 1.0
+        args = (wl.kv_cache, wl.req_to_token, wl.req_pool_indices, wl.cache_seqlens, wl.softmax_scale,
+                wl.causal)
+        o8, l8 = oracle.mla_decode(codes, *args, kv_is_fp8=wl.is_fp8, descale_q=scale, descale_k=dk,
+                                   q_is_fp8=True)
+        ob, lb = oracle.mla_decode(vals, *args, kv_is_fp8=wl.is_fp8, descale_q=scale, descale_k=dk)
+        assert np.array_equal(o8, ob) and np.array_equal(l8, lb)
+        # and the scale really enters: descale_q = 2 * scale doubles every score
+        o2, l2 = oracle.mla_decode(codes, *args, kv_is_fp8=wl.is_fp8, descale_q=2 * scale,
+                                   descale_k=dk, q_is_fp8=True)
+        assert not np.allclose(l2, l8)
+
+
 def test_empty_and_fully_masked_rows():
     wl = W.make_case([0, 3], h=2, seed=16)
     o, lse = run_oracle(wl)
