@@ -14,8 +14,12 @@ Reported (one JSON line on rank 0):
   roofline     the attention call (decode kernel + merge) against the measured HBM peak:
                algorithmic (KV + Q) bytes / its CUDA-event time;
   e2e          the same metric through the public API with the step's inputs (q,
-               seq_lens, req_pool_indices) copied from pinned host memory and the
-               outputs (o, lse) copied back inside the timed region;
+               seq_lens, cache_seqlens, req_pool_indices) copied from pinned host memory and
+               the outputs (o, lse) copied back inside the timed region, the copies of
+               neighbouring steps overlapping the step's compute on their own streams;
+  per_config   every workload (tiny, DeepSeek-V3 decode, skewed long context, fp8 cache,
+               target-verify): us per call, metadata us, roofline and clocks, from a short
+               timed run each;
   cpu_baseline the CPU fp64 oracle on a bounded sample of the same workload (rank 0, N=1).
 Multi-GPU: independent replicas (the path has no exchange step); NCCL is used only for
 the barrier and the max-over-ranks reduction of the timings.
@@ -55,6 +59,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the --config workload")
+    ap.add_argument("--per-config-steps", type=int, default=50,
+                    help="timed steps of each other workload in the per_config entries")
     return ap.parse_args(argv)
 
 
@@ -115,31 +123,33 @@ def captured_traffic(config):
 
 
 def roofline_entry(kv_bytes, q_bytes, flops, attn_s, peaks, peak_src, is_fp8, traffic):
-    """The bench line's roofline object for one attention call of attn_s seconds: bound by HBM
-    (algorithmic KV + Q bytes) or by the tensor cores (algorithmic FLOPs at the measured bf16
-    peak; the e4m3 cache computes with f16 MMAs, whose peak is the bf16 one).  An e4m3 cache is
-    also reported against the fp8 peak (the measured bf16 peak x the nominal fp8 / bf16 ratio 2),
-    the rate a path with fp8 MMAs would have."""
+    """The bench line's roofline object for one attention call of attn_s seconds: the slower of
+    the algorithmic KV + Q bytes at the measured HBM bandwidth and the algorithmic FLOPs at the
+    dense tensor peak of the cache's precision -- the measured bf16 peak for a bf16 cache, the
+    fp8 peak (the measured bf16 peak x the nominal fp8 / bf16 ratio 2) for an e4m3 cache.  An
+    e4m3 cache is also reported against the bf16 peak, the rate of the f16 MMAs it runs."""
+    tensor_peak = peaks["bf16_tflops"] * (2.0 if is_fp8 else 1.0)
     t_hbm = (kv_bytes + q_bytes) / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_tc = flops / (tensor_peak * 1e12)
     achieved_gbs = (kv_bytes + q_bytes) / attn_s / 1e9
     achieved_tf = flops / attn_s / 1e12
     if t_hbm >= t_tc:
         roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"]}
     else:
-        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved_tf / tensor_peak}
     roof.update({"traffic": traffic, "traffic_unit": "bytes per launch",
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
                  if peak_src == "measured" else "fallback",
                  "kernel": "mla_decode_paged call (decode kernel + split merge)",
                  "roofline_time_us": max(t_hbm, t_tc) * 1e6,
-                 "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s})
+                 "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s,
+                 "tensor_peak_dtype": "fp8" if is_fp8 else "bf16"})
     if is_fp8:
-        fp8_peak = 2.0 * peaks["bf16_tflops"]
-        roof.update({"fp8_peak_tflops": fp8_peak, "frac_of_fp8_peak": achieved_tf / fp8_peak,
-                     "fp8_peak_source": "measured bf16 peak x 2 (nominal fp8 / bf16 ratio)"})
+        roof.update({"tensor_peak_tflops": tensor_peak,
+                     "tensor_peak_source": "measured bf16 peak x 2 (nominal fp8 / bf16 ratio)",
+                     "frac_of_bf16_peak": achieved_tf / peaks["bf16_tflops"]})
     return roof
 
 
@@ -316,12 +326,201 @@ def run_reference(args):
     return 0
 
 
+class Case:
+    """One workload resident on the device, with its metadata / attention steps captured as
+    CUDA graphs the way a serving engine replays them."""
+
+    def __init__(self, cfg, seed, dev, flush_mb):
+        import torch
+        import paged_kv_mla_create_b200 as mla
+        from paged_kv_mla_create_b200 import workloads as W
+        self.mla, self.dev, self.cfg = mla, dev, cfg
+        self.host = host = W.make_workload(cfg, seed=seed)
+        self.wl = host.to(dev)
+        self.kv_bytes, self.q_bytes, self.flops = algorithmic(host)
+        bs, q_len, h = host.bs, host.q_len, host.h
+        self.parts = mla.num_sm_parts(q_len * h, 1, mla.sm_count(dev))
+        self.bt = torch.empty((bs, host.max_pages), dtype=torch.int32, device=dev)
+        self.md = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
+        self.ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
+        self.o = torch.empty((bs, q_len, h, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((bs, q_len, h), dtype=torch.float32, device=dev)
+        self.ws = torch.empty((mla.workspace_bytes(bs, q_len, h, self.parts),), dtype=torch.uint8,
+                              device=dev)
+        self.flush = torch.empty((flush_mb << 20,), dtype=torch.uint8, device=dev)
+        self.flush_rd = torch.ones((flush_mb << 20,), dtype=torch.uint8, device=dev)
+        self.side = torch.cuda.Stream(dev)
+
+    def flush_l2(self, i):
+        self.flush.fill_(i & 0xFF)
+        self.flush_rd.max()   # evicts the written lines while still outside the timed region
+
+    def metadata(self, w):
+        import torch
+        host = self.host
+        # the page table and the plan are independent: the plan runs on a side stream
+        cur = torch.cuda.current_stream(self.dev)
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            self.mla.get_mla_metadata(w.cache_seqlens, host.q_len * host.h, 1, host.is_fp8,
+                                      out=(self.md, self.ns))
+        self.mla.build_block_table(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
+                                   seq_len_add=host.num_draft_tokens, out=self.bt)
+        cur.wait_stream(self.side)
+
+    def attention(self, w, o=None, lse=None):
+        host = self.host
+        self.mla.mla_decode_paged(w.q, w.kv_cache, self.bt, w.cache_seqlens, 512, self.md, self.ns,
+                                  host.softmax_scale, host.causal, w.descale_q, w.descale_k,
+                                  out=self.o if o is None else o, lse=self.lse if lse is None else lse,
+                                  workspace=self.ws)
+
+    def capture(self):
+        import torch
+        stream = torch.cuda.current_stream(self.dev)
+        cap = torch.cuda.Stream(self.dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            self.metadata(self.wl)
+            self.attention(self.wl)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize(self.dev)
+        self.g_meta, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_meta):
+            self.metadata(self.wl)
+        with torch.cuda.graph(self.g_attn):
+            self.attention(self.wl)
+
+    def release(self):
+        for name in ("g_meta", "g_attn"):
+            if hasattr(self, name):
+                delattr(self, name)
+
+    def time_steps(self, steps, warmup, world, clocks=None):
+        """Warm-up, then `steps` timed graph replays (L2 flushed before each, outside its
+        events).  Returns (step_ms, attn_ms, meta_ms, clock record)."""
+        import torch
+        import torch.distributed as dist
+        for i in range(warmup):
+            self.flush_l2(i)
+            self.metadata(self.wl)
+            self.attention(self.wl)
+        torch.cuda.synchronize(self.dev)
+        if self.mla.read_device_error(self.dev) != 0:
+            raise RuntimeError("device error word set during warm-up")
+        self.capture()
+        for i in range(3):
+            self.flush_l2(i)
+            self.g_meta.replay()
+            self.g_attn.replay()
+        torch.cuda.synchronize(self.dev)
+        stream = torch.cuda.current_stream(self.dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(self.dev)
+        if clocks is not None:
+            clocks.start()
+        for k in range(steps):
+            self.flush_l2(k)
+            ev[k][0].record(stream)
+            self.g_meta.replay()
+            ev[k][1].record(stream)
+            self.g_attn.replay()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize(self.dev)
+        if world > 1:
+            dist.barrier()
+        clk = clocks.stop() if clocks is not None else None
+        self.release()
+        step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / steps
+        attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        meta_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        return step_ms, attn_ms, meta_ms, clk
+
+    def time_e2e(self, steps):
+        """The same step end to end through the public API, from pinned host buffers: step k's
+        inputs (q, seq_lens, cache_seqlens, req_pool_indices) are copied in on a copy stream
+        while step k - 1 computes, and step k's o and lse are copied out on another while step
+        k + 1 computes (two device buffer sets).  Every step's copies lie inside the timed
+        region, which runs from the first copy in to the last copy out.  No L2 flush: the KV
+        cache every step streams is larger than L2.  Returns (ms per step, h2d, d2h bytes)."""
+        import dataclasses
+        import torch
+        host, wl, dev = self.host, self.wl, self.dev
+        pin = [t.pin_memory() for t in (host.q, host.seq_lens, host.cache_seqlens,
+                                        host.req_pool_indices)]
+        outs_h = [(torch.empty(self.o.shape, dtype=self.o.dtype, pin_memory=True),
+                   torch.empty(self.lse.shape, dtype=self.lse.dtype, pin_memory=True)) for _ in range(2)]
+        ins_d, outs_d, wls = [], [], []
+        for _ in range(2):
+            d = [torch.empty_like(t, device=dev) for t in pin]
+            ins_d.append(d)
+            outs_d.append((torch.empty_like(self.o), torch.empty_like(self.lse)))
+            wls.append(dataclasses.replace(wl, q=d[0], seq_lens=d[1], cache_seqlens=d[2],
+                                           req_pool_indices=d[3]))
+        h2d = sum(t.numel() * t.element_size() for t in pin)
+        d2h = sum(t.numel() * t.element_size() for t in outs_h[0])
+        comp = torch.cuda.current_stream(dev)
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def run(n, timed):
+            torch.cuda.synchronize(dev)
+            if timed:
+                t0.record(comp)
+            s_in.wait_stream(comp)
+            s_out.wait_stream(comp)
+            for k in range(n):
+                j = k & 1
+                if k >= 2:
+                    s_in.wait_event(ev_comp[j])      # step k - 2 is done with input set j
+                with torch.cuda.stream(s_in):
+                    for dst, src in zip(ins_d[j], pin):
+                        dst.copy_(src, non_blocking=True)
+                    ev_in[j].record(s_in)
+                comp.wait_event(ev_in[j])
+                if k >= 2:
+                    comp.wait_event(ev_out[j])       # step k - 2's outputs have left set j
+                self.metadata(wls[j])
+                self.attention(wls[j], o=outs_d[j][0], lse=outs_d[j][1])
+                ev_comp[j].record(comp)
+                s_out.wait_event(ev_comp[j])
+                with torch.cuda.stream(s_out):
+                    outs_h[j][0].copy_(outs_d[j][0], non_blocking=True)
+                    outs_h[j][1].copy_(outs_d[j][1], non_blocking=True)
+                    ev_out[j].record(s_out)
+            comp.wait_stream(s_out)
+            comp.wait_stream(s_in)
+            if timed:
+                t1.record(comp)
+            torch.cuda.synchronize(dev)
+
+        run(4, False)
+        run(steps, True)
+        return t0.elapsed_time(t1) / steps, h2d, d2h
+
+
+def config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src):
+    from paged_kv_mla_create_b200.workloads import CONFIGS
+    attn_s = attn_ms * 1e-3
+    return {"workload": CONFIGS[case.cfg]["name"], "us_per_call": attn_ms * 1e3,
+            "metadata_us": meta_ms * 1e3, "us_per_step": step_ms * 1e3,
+            "kv_gbs_per_call": case.kv_bytes / attn_s / 1e9, "tflops": case.flops / attn_s / 1e12,
+            "kv_bytes": case.kv_bytes, "q_bytes": case.q_bytes, "flops": case.flops,
+            "roofline": roofline_entry(case.kv_bytes, case.q_bytes, case.flops, attn_s, peaks,
+                                       peak_src, case.host.is_fp8, captured_traffic(case.cfg)),
+            "clocks": clk}
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
 
     import paged_kv_mla_create_b200 as mla
-    from paged_kv_mla_create_b200 import workloads as W
 
     rank, world, local = dist_env()
     if world > 1:
@@ -332,139 +531,40 @@ def run_b200(args):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     mla.library()
+    peaks, peak_src = load_peaks()
 
-    host = W.make_workload(args.config, seed=replica_seed(args.config, rank))
-    wl = host.to(dev)
-    kv_bytes, q_bytes, flops = algorithmic(host)
-    bs, q_len, h = host.bs, host.q_len, host.h
-    parts = mla.num_sm_parts(q_len * h, 1, mla.sm_count(dev))
-    bt = torch.empty((bs, host.max_pages), dtype=torch.int32, device=dev)
-    md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
-    ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
-    o = torch.empty((bs, q_len, h, 512), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((bs, q_len, h), dtype=torch.float32, device=dev)
-    ws = torch.empty((mla.workspace_bytes(bs, q_len, h, parts),), dtype=torch.uint8, device=dev)
-    flush = torch.empty((args.flush_mb << 20,), dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones((args.flush_mb << 20,), dtype=torch.uint8, device=dev)
-
-    def flush_l2(i):
-        flush.fill_(i & 0xFF)
-        flush_rd.max()   # evicts the written lines while still outside the timed region
-
-    side = torch.cuda.Stream(dev)
-
-    def metadata(w):
-        # the page table and the plan are independent: the plan runs on a side stream
-        cur = torch.cuda.current_stream(dev)
-        side.wait_stream(cur)
-        with torch.cuda.stream(side):
-            mla.get_mla_metadata(w.cache_seqlens, q_len * h, 1, host.is_fp8, num_parts=parts,
-                                 out=(md, ns))
-        mla.build_block_table(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
-                              seq_len_add=host.num_draft_tokens, out=bt)
-        cur.wait_stream(side)
-
-    def attention(w):
-        mla.mla_decode_paged(w.q, w.kv_cache, bt, w.cache_seqlens, 512, md, ns,
-                             host.softmax_scale, host.causal, w.descale_q, w.descale_k,
-                             out=o, lse=lse, workspace=ws)
-
-    stream = torch.cuda.current_stream(dev)
-    for i in range(args.warmup):
-        flush_l2(i)
-        metadata(wl)
-        attention(wl)
-    torch.cuda.synchronize(dev)
-    if mla.read_device_error(dev) != 0:
-        raise RuntimeError("device error word set during warm-up")
-
-    # The step as a serving engine runs it: both parts captured once as CUDA graphs and
-    # replayed (the calls allocate nothing and never synchronise, so they capture as is).
-    g_meta, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream(dev)
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        metadata(wl)
-        attention(wl)
-    stream.wait_stream(cap)
-    torch.cuda.synchronize(dev)
-    with torch.cuda.graph(g_meta):
-        metadata(wl)
-    with torch.cuda.graph(g_attn):
-        attention(wl)
-    for i in range(3):
-        flush_l2(i)
-        g_meta.replay()
-        g_attn.replay()
-    torch.cuda.synchronize(dev)
-
+    case = Case(args.config, replica_seed(args.config, rank), dev, args.flush_mb)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     clocks = ClockSampler(gpu_id_for(dev))
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    for k in range(K):
-        flush_l2(k)
-        ev[k][0].record(stream)
-        g_meta.replay()
-        ev[k][1].record(stream)
-        g_attn.replay()
-        ev[k][2].record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    del g_meta, g_attn
-    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / K
-    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    meta_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-
-    # end to end through the public API, host buffers in and out
-    pin_q = host.q.pin_memory()
-    pin_sl = host.seq_lens.pin_memory()
-    pin_cl = host.cache_seqlens.pin_memory()
-    pin_rpi = host.req_pool_indices.pin_memory()
-    out_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    out_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    dq = torch.empty_like(wl.q)
-    dsl = torch.empty_like(wl.seq_lens)
-    dcl = torch.empty_like(wl.cache_seqlens)
-    drpi = torch.empty_like(wl.req_pool_indices)
-    import dataclasses
-    we = dataclasses.replace(wl, q=dq, seq_lens=dsl, cache_seqlens=dcl, req_pool_indices=drpi)
-    h2d = sum(t.numel() * t.element_size() for t in (pin_q, pin_sl, pin_cl, pin_rpi))
-    d2h = out_o.numel() * out_o.element_size() + out_lse.numel() * out_lse.element_size()
-    KE = max(1, min(args.e2e_steps, K))
-    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(KE)]
-    torch.cuda.synchronize(dev)
-    for k in range(KE):
-        flush_l2(k)
-        ee[k][0].record(stream)
-        dq.copy_(pin_q, non_blocking=True)
-        dsl.copy_(pin_sl, non_blocking=True)
-        dcl.copy_(pin_cl, non_blocking=True)
-        drpi.copy_(pin_rpi, non_blocking=True)
-        metadata(we)
-        attention(we)
-        out_o.copy_(o, non_blocking=True)
-        out_lse.copy_(lse, non_blocking=True)
-        ee[k][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in ee) / KE
+    step_ms, attn_ms, meta_ms, clk = case.time_steps(K, args.warmup, world, clocks)
+    e2e_ms, h2d, d2h = case.time_e2e(max(1, min(args.e2e_steps, K)))
     err = mla.read_device_error(dev)
-
     step_ms, attn_ms, meta_ms, e2e_ms, err = reduce_max_over_ranks(
         [step_ms, attn_ms, meta_ms, e2e_ms, float(err)], dev, world)
     if err:
         raise RuntimeError(f"device error word {int(err)} after the timed run")
+    head = config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src)
+    host = case.host
+    kv_bytes = case.kv_bytes
+    del case
+    torch.cuda.empty_cache()
 
-    peaks, peak_src = load_peaks()
-    attn_s = attn_ms * 1e-3
-    achieved_tf = flops / attn_s / 1e12
-    roof = roofline_entry(kv_bytes, q_bytes, flops, attn_s, peaks, peak_src, host.is_fp8,
-                          captured_traffic(args.config))
+    # every other workload, with a short timed run each (its own clock record)
+    per_config = {str(args.config): head}
+    if not args.no_per_config:
+        for cfg in (1, 2, 3, 4, 5):
+            if cfg == args.config:
+                continue
+            c = Case(cfg, replica_seed(cfg, rank), dev, args.flush_mb)
+            sm, am, mm, ck = c.time_steps(max(1, min(K, args.per_config_steps)), max(3, min(args.warmup, 5)),
+                                          world, ClockSampler(gpu_id_for(dev)))
+            e = mla.read_device_error(dev)
+            sm, am, mm, e = reduce_max_over_ranks([sm, am, mm, float(e)], dev, world)
+            if e:
+                raise RuntimeError(f"device error word {int(e)} after workload {cfg}")
+            per_config[str(cfg)] = config_entry(c, sm, am, mm, ck, peaks, peak_src)
+            del c
+            torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:
@@ -477,14 +577,17 @@ def run_b200(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f16" if host.is_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(args.config, host, world, args.flush_mb),
-        "us_per_call": attn_ms * 1e3, "metadata_us": meta_ms * 1e3,
-        "kv_gbs_per_call": kv_bytes / attn_s / 1e9, "tflops": achieved_tf,
-        "tensor_frac": achieved_tf / peaks["bf16_tflops"],
-        "roofline": roof,
+        "us_per_call": head["us_per_call"], "metadata_us": head["metadata_us"],
+        "kv_gbs_per_call": head["kv_gbs_per_call"], "tflops": head["tflops"],
+        "tensor_frac": head["tflops"] / peaks["bf16_tflops"],
+        "roofline": head["roofline"],
         "e2e": {"value": job_value(world, kv_bytes, e2e_ms), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "overlap": "inputs of step k+1 copied in and outputs of step k-1 copied out on "
+                           "their own streams while step k computes"},
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clk,
+        "per_config": per_config,
     }
     if world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(host, args.cpu_seconds)

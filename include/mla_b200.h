@@ -70,7 +70,9 @@ enum {
     MLA_DEVERR_LEN_OUT_OF_RANGE = 4,   /* a length exceeds the table / req_to_token width: clamped     */
     MLA_DEVERR_BAD_METADATA = 8,       /* a scheduler row is not a valid cursor range: part skipped    */
     MLA_DEVERR_WAIT_TIMEOUT = 16,      /* a pipeline wait exceeded its bound: the CTA gave up          */
-    MLA_DEVERR_Q_RANGE = 32            /* e4m3 cache: a q value beyond the f16 range (|q| > 65504)     */
+    MLA_DEVERR_Q_RANGE = 32,           /* e4m3 cache: a q value beyond the f16 range (|q| > 65504)     */
+    MLA_DEVERR_SLOT_INVALID = 64       /* page table: a req_to_token slot read for page p is negative    */
+                                       /* (entry -1) or not the first slot of a page (slot % 64 != 0)  */
 };
 
 typedef struct CUstream_st* mla_stream_t;  /* identical to cudaStream_t */
@@ -93,7 +95,8 @@ MLA_API int32_t mla_abi_version(void);
  * (the pool viewed [-1, page_size, 1, 576] puts slots page_size*P .. page_size*P+page_size-1
  * in page P, so slots must be page-aligned and in order inside a page).
  * Entries p in [cdiv(L_b, page_size), max_pages) are written with -1 when fill_tail != 0
- * and left untouched otherwise (the caller's pre-fill, as in the graph-capture path).
+ * and left untouched otherwise (the caller's pre-fill, as in the graph-capture path, which
+ * fills its table with 1); columns from max_pages to block_table_stride are never touched.
  *
  *   req_to_token         int32 [req_to_token_rows, req_to_token_stride] (row-major)
  *   req_pool_indices     [bs], int32 or int64 (rpi_dtype)
@@ -102,7 +105,10 @@ MLA_API int32_t mla_abi_version(void);
  *   page_size            must be 64
  * Device checks: a row index outside [0, req_to_token_rows) leaves the row at -1 and
  * sets MLA_DEVERR_ROW_OUT_OF_RANGE; L_b beyond max_pages pages or beyond
- * req_to_token_stride positions is clamped and sets MLA_DEVERR_LEN_OUT_OF_RANGE.
+ * req_to_token_stride positions is clamped and sets MLA_DEVERR_LEN_OUT_OF_RANGE; a slot
+ * read for page p that is not page-aligned (slot % 64 != 0: the request's slots are not
+ * whole pages in order) still gives slot / 64 but sets MLA_DEVERR_SLOT_INVALID, and a
+ * negative slot gives -1 and sets the same bit.
  */
 MLA_API mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t req_to_token_rows,
                                    int64_t req_to_token_stride, const void* req_pool_indices,
@@ -123,8 +129,11 @@ MLA_API mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t 
 MLA_API int32_t mla_num_sm_parts(int32_t sm_count, int32_t num_heads_per_head_k, int32_t num_heads_k);
 
 /*
- * Split-KV scheduler (flashmla_backend.py, get_mla_metadata: tile_scheduler_metadata
+ * Split-KV scheduler (flashmla_backend.py, get_mla_metadata(cache_seqlens,
+ * num_heads_per_head_k, num_heads_k, is_fp8_kvcache) returning tile_scheduler_metadata
  * int32 [num_sm_parts, 8], num_sm_parts <= the SM count, and num_splits int32 [bs+1]).
+ * The part count is num_sm_parts = mla_num_sm_parts(sm_count, num_heads_per_head_k,
+ * num_heads_k); the caller sizes tile_scheduler_metadata with the same call.
  * The pages fix only these shapes; the contents are defined here:
  *   blocks_b = cdiv(cache_seqlens[b], 64); each piece of a request costs its blocks plus
  *   a fixed overhead of 5 blocks; total = sum_b (blocks_b + 5); every part has the budget
@@ -138,14 +147,17 @@ MLA_API int32_t mla_num_sm_parts(int32_t sm_count, int32_t num_heads_per_head_k,
  * Every block of every request is covered exactly once within num_sm_parts parts, and
  * num_splits[bs] <= bs + num_sm_parts - 1.
  *   cache_seqlens          int32 [bs] (negative lengths count as 0)
- *   num_sm_parts           from mla_num_sm_parts (>= 1)
+ *   num_heads_per_head_k   q_len * h_q (num_draft_tokens * h_q in target-verify), > 0
+ *   num_heads_k            1 for MLA, > 0
  *   is_fp8_kvcache         accepted; it does not change the plan
- *   tile_scheduler_metadata int32 [num_sm_parts, 8] (written)
+ *   sm_count               SMs of the device the attention runs on, > 0
+ *   tile_scheduler_metadata int32 [num_sm_parts, 8] (written), 16-byte aligned
  *   num_splits             int32 [bs + 1] (written)
  * One single-CTA launch; bs must be <= 1,048,576.
  */
 MLA_API mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
-                                  int32_t num_sm_parts, int32_t is_fp8_kvcache,
+                                  int32_t num_heads_per_head_k, int32_t num_heads_k,
+                                  int32_t is_fp8_kvcache, int32_t sm_count,
                                   int32_t* tile_scheduler_metadata, int32_t* num_splits,
                                   mla_stream_t stream);
 
@@ -170,11 +182,14 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *   lse = ln sum_j exp(s_j);  o = sum_j exp(s_j - lse) v_j.
  *   A row with no allowed key gets o = 0 and lse = -inf.
  *   Arithmetic: S in fp32 from bf16 products (bf16 cache) or f16 products (e4m3 cache:
- *   e4m3 values and bf16 q values are exact in f16, so q must lie within f16's range,
- *   |q| <= 65504, or MLA_DEVERR_Q_RANGE is recorded and o is undefined); P rounded to
- *   bf16 (f16 with an e4m3 cache) for the P V product; O accumulated in fp32.
+ *   every e4m3 value is exact in f16; a bf16 q value is exact in f16 when its magnitude
+ *   lies in [2^-14, 65504] or it is zero, while magnitudes in [2^-24, 2^-14) keep only
+ *   the bits of an f16 subnormal and smaller ones round to zero, an error far below the
+ *   attention tolerance; |q| > 65504 records MLA_DEVERR_Q_RANGE and o is undefined); P
+ *   rounded to bf16 (f16 with an e4m3 cache) for the P V product; O accumulated in fp32.
  *
- *   q                 bf16 [bs, q_len, h_q, head_dim], contiguous
+ *   q                 bf16 [bs, q_len, h_q, head_dim], contiguous; q_len * h_q must not
+ *                     exceed 65535 * 128 (MLA_ERR_UNSUPPORTED)
  *   q_dtype           MLA_DTYPE_BF16
  *   head_dim          576 (kv_lora_rank 512 + qk_rope_head_dim 64); head_dim_v 512
  *   k_cache           [num_pages, page_size, head_dim] bf16 or e4m3 (kv_dtype), contiguous;
@@ -189,7 +204,9 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *   softmax_scale     host float (1/sqrt(192) for DeepSeek-V3)
  *   causal            0 or 1
  *   descale_q, descale_k  device fp32 [1]; NULL means 1.0.  descale_k scales the fp8
- *                     cache values; descale_q scales q.
+ *                     cache values and must be NULL with a bf16 cache (the backend passes
+ *                     the descales only with an fp8 cache), else MLA_ERR_INVALID_ARG;
+ *                     descale_q scales q.
  *   out               bf16 [bs, q_len, h_q, 512] (written)
  *   lse               fp32 [bs, q_len, h_q] natural-log log-sum-exp (written)
  *   workspace         at least mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts)

@@ -68,7 +68,7 @@ def library() -> ctypes.CDLL:
     lib.mla_build_block_table.restype = I32
     lib.mla_num_sm_parts.argtypes = [I32, I32, I32]
     lib.mla_num_sm_parts.restype = I32
-    lib.mla_get_mla_metadata.argtypes = [P, I32, I32, I32, P, P, P]
+    lib.mla_get_mla_metadata.argtypes = [P, I32, I32, I32, I32, I32, P, P, P]
     lib.mla_get_mla_metadata.restype = I32
     lib.mla_decode_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.mla_decode_workspace_bytes.restype = SZ
@@ -153,22 +153,34 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, num_heads_per_head_k: int,
                      num_heads_k: int = 1, is_fp8_kvcache: bool = False,
                      num_parts: Optional[int] = None,
                      out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
-    """(tile_scheduler_metadata int32 [num_sm_parts, 8], num_splits int32 [bs + 1])."""
+    """(tile_scheduler_metadata int32 [num_sm_parts, 8], num_splits int32 [bs + 1]).
+
+    The part count follows from the device's SM count; ``num_parts`` plans for that many
+    parts instead (the SM count of a device with 2 SMs per part and query tile)."""
     _require_cuda(cache_seqlens)
     if cache_seqlens.dtype != torch.int32:
         raise ValueError("cache_seqlens must be int32 (the backend casts with .to(torch.int32))")
+    if num_heads_per_head_k <= 0 or num_heads_k <= 0:
+        raise ValueError("num_heads_per_head_k and num_heads_k must be positive")
     sl = cache_seqlens.contiguous()
     bs = int(sl.shape[0])
     dev = sl.device
-    parts = num_parts if num_parts is not None else num_sm_parts(num_heads_per_head_k, num_heads_k,
-                                                                 sm_count(dev))
+    if num_parts is not None:
+        m_tiles = -(-num_heads_per_head_k // 128)
+        sms = 2 * m_tiles * num_heads_k * int(num_parts)
+    else:
+        sms = sm_count(dev)
+    parts = num_sm_parts(num_heads_per_head_k, num_heads_k, sms)
     if out is None:
         md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
         ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
     else:
         md, ns = out
-    _check(library().mla_get_mla_metadata(_ptr(sl), bs, parts, int(bool(is_fp8_kvcache)),
-                                          _ptr(md), _ptr(ns), _stream(dev)),
+        if md.shape[0] != parts or ns.numel() != bs + 1:
+            raise ValueError("out tensors do not match the plan's shapes")
+    _check(library().mla_get_mla_metadata(_ptr(sl), bs, int(num_heads_per_head_k), int(num_heads_k),
+                                          int(bool(is_fp8_kvcache)), sms, _ptr(md), _ptr(ns),
+                                          _stream(dev)),
            "mla_get_mla_metadata")
     return md, ns
 

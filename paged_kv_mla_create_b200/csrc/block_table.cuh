@@ -41,7 +41,9 @@ build_block_table_kernel(const int32_t* __restrict__ req_to_token, int64_t r2t_r
     int32_t* dst = block_table + b * bt_stride + p;
     if (p < npages) {
         const int32_t slot = __ldg(req_to_token + row * r2t_stride + static_cast<int64_t>(p) * kPage);
-        // Slots are non-negative; floor division maps a slot to its page.
+        // Slots are non-negative and page-aligned at the start of each page (the pool viewed
+        // [-1, 64, 1, 576] holds a page's 64 slots in order); division maps a slot to its page.
+        if (slot < 0 || (slot & (kPage - 1)) != 0) raise_error(64 /* MLA_DEVERR_SLOT_INVALID */);
         *dst = slot >= 0 ? slot / kPage : -1;
     } else if (fill_tail) {
         *dst = -1;

@@ -46,7 +46,7 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
     // A request of few pieces drops its rows' L2 lines once merged (they need no write-back);
     // the loads of a many-piece request (a long serial loop here) only lower their L2
     // priority, which measured faster than dropping each line.
-    const bool discard = MLA_L2_HINTS && n <= kDiscardMaxPieces;
+    const bool discard = n <= kDiscardMaxPieces;
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
@@ -63,8 +63,7 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
                 const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    v[j][k] = (MLA_L2_HINTS && !discard) ? ld_global_nc_v4_hint(src + lane + 32 * k, read_pol)
-                                                         : __ldg(src + lane + 32 * k);
+                    v[j][k] = discard ? __ldg(src + lane + 32 * k) : ld_global_nc_v4_hint(src + lane + 32 * k, read_pol);
             } else {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) v[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -49,31 +49,6 @@
 namespace mla {
 namespace decode {
 
-// Optional pipeline trace (compiled only with -DMLA_TRACE): SM clock at each pipeline
-// event of the first kTraceTiles tiles of cluster 0, query tile 0.
-#ifdef MLA_TRACE
-constexpr int kTraceTiles = 64, kTraceEvents = 32;
-__device__ long long g_trace[2][kTraceTiles][kTraceEvents];
-__device__ unsigned long long g_ctatrace[1024][16];
-#define MLA_CTA_EVENT(ev)                                                                 \
-    do {                                                                                  \
-        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                             \
-        if (cta_ < 1024 && (ev) < 16) g_ctatrace[cta_][(ev)] = global_timer_ns();         \
-    } while (0)
-#define MLA_TRACE_EVENT(tile, ev)                                                         \
-    do {                                                                                  \
-        if (blockIdx.x < 2 && blockIdx.y == 0 && (tile) < (uint32_t)kTraceTiles)          \
-            g_trace[blockIdx.x][(tile)][(ev)] = clock64();                                \
-    } while (0)
-#else
-#define MLA_CTA_EVENT(ev) \
-    do {                  \
-    } while (0)
-#define MLA_TRACE_EVENT(tile, ev) \
-    do {                          \
-    } while (0)
-#endif
-
 constexpr int kRows = 128;                 // query rows per tile (both CTAs)
 constexpr int kCtaRows = 64;               // query rows per CTA
 constexpr int kPage = 64;                  // tokens per page
@@ -87,60 +62,6 @@ constexpr int kQHiChunks = kChunks - kQLoChunks;   // Q columns [256, 576): shar
 constexpr int kQHiBytes = kQHiChunks * kBox;       // 40 KB
 constexpr int kKSlots = 2;                 // K ring: two tiles
 constexpr int kKSlotBytes = kChunks * kBox;        // 72 KB: one page, all 576 columns
-#ifndef MLA_KOPS
-#define MLA_KOPS 1
-#endif
-#ifndef MLA_V_TMA
-#define MLA_V_TMA 1
-#endif
-// Measured alternatives, kept selectable: the page loaded in three 24 KB pieces by three
-// warps (S starting on the first piece), and the bf16 partner V through registers like the
-// e4m3 one, were each slower on B200 than one 72 KB load and a TMA load of the partner V
-// (the SM's TMA unit and its global loads share one path; more, smaller requests cost more).
-#ifndef MLA_L2_PREFETCH
-#define MLA_L2_PREFETCH 0
-#endif
-// A K warp that has issued its tile's page load asks the L2, through the load/store path,
-// for the page of its next tile (two tiles on), so that load finds the page in L2.  (A TMA
-// prefetch would queue in the same TMA unit as the loads, which measured slower.)
-constexpr bool kL2Prefetch = MLA_L2_PREFETCH != 0;
-#ifndef MLA_P_SIGNAL_ONCE
-#define MLA_P_SIGNAL_ONCE 0
-#endif
-#ifndef MLA_P_SIGNAL_ASYNC
-#define MLA_P_SIGNAL_ASYNC 1
-#endif
-// The peer CTA's softmax warps signal "P written" to the leader's barrier: each warp with a
-// remote release arrive (0), or once per CTA after a local barrier (1); or (async) each warp
-// with a 4-byte st.async into the leader whose complete_tx lands on the barrier, ordered
-// after the warp's P stores by its fence.proxy.async, while the leader's warps arrive with
-// expect_tx (a remote release arrive measured ~1000 cycles before the leader saw it).
-constexpr bool kPSignalOnce = MLA_P_SIGNAL_ONCE != 0;
-constexpr bool kPSignalAsync = MLA_P_SIGNAL_ASYNC != 0 && !kPSignalOnce;
-#ifndef MLA_SIGNAL_ALL
-#define MLA_SIGNAL_ALL 1
-#endif
-// Also "Q written" (after the warp's tensor-memory stores completed) and "S / O read" (after
-// its tensor-memory loads completed) from the peer by st.async; the data is already in place
-// (or already read) when the signal is sent, so a 4-byte complete_tx is all the leader needs.
-constexpr bool kSignalAll = MLA_SIGNAL_ALL != 0;
-#ifndef MLA_ISSUER_POLL_CTA
-#define MLA_ISSUER_POLL_CTA 1
-#endif
-// The MMA issuer's barrier tests acquire at CTA scope (1) or cluster scope (0); the data
-// behind a barrier the peer completes is ordered by the peer's fence.proxy.async and the
-// st.async / TMA complete_tx itself, and the CTA-scope test measured ~1% faster.
-constexpr bool kIssuerPollCta = MLA_ISSUER_POLL_CTA != 0;
-constexpr int kKOps = MLA_KOPS;            // bf16 page load in kKOps pieces of 9 / kKOps chunks
-constexpr int kKOpChunks = kChunks / kKOps;
-constexpr bool kVTma = MLA_V_TMA != 0;     // bf16 partner V by TMA (else through registers)
-static_assert(kKOps == 1 || kKOps == 3, "page pieces");
-// KV page loads evict-first and split partials evict-last in L2, so that the partials are still
-// in L2 when the merge reads them (the merge then drops their lines without a write-back).
-constexpr bool kL2Hints = MLA_L2_HINTS != 0;
-#ifndef MLA_KV_EVICT_FIRST
-#define MLA_KV_EVICT_FIRST 1
-#endif
 constexpr int kPBytes = 2 * kBox;          // P: 64 rows x 128 tokens bf16
 constexpr int kThreads = 384;              // 12 warps (roles above)
 constexpr int kSoftmaxWarp0 = 4;
@@ -165,10 +86,10 @@ constexpr int kOffBar = kOffPSig + 128;   // landing words: P 0..3, V 4..7, K 8,
                                             // S read 16..19, O read 20..23
 
 enum : int {
-    kBarKFull = 0,                      // leader (x slots x pieces): both CTAs' piece j landed
-    kBarKEmpty = kBarKFull + kKSlots * kKOps,   // both: the tile's PV finished (slot reusable)
+    kBarKFull = 0,                      // leader (x slots): both CTAs' pages of the tile landed
+    kBarKEmpty = kBarKFull + kKSlots,   // both: the tile's PV finished (slot reusable)
     kBarQKDone = kBarKEmpty + kKSlots,  // both: the tile's S MMAs finished reading the slot
-    kBarVFull = kBarQKDone + kKSlots,   // leader: the 8 Q warps stored the partner V
+    kBarVFull = kBarQKDone + kKSlots,   // leader: the pair's partner V landed
     kBarQFull = kBarVFull + kKSlots,    // leader: Q columns [256, 576) landed (tx) + eight
                                         // warps wrote Q columns [0, 256) to tensor memory
     kBarQEmpty,                         // both: the unit's last S MMA finished (Q reusable)
@@ -180,7 +101,6 @@ enum : int {
     kBarOEmpty,                         // leader: 8 softmax warps read O out
     kBarXchg,                           // local (x2): the 128 softmax threads posted row maxima
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
-    kBarPLocal,                         // local: this CTA's 4 softmax warps wrote P (peer CTA)
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
 };
@@ -349,39 +269,27 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int part = blockIdx.x >> 1;
     const int mtile = blockIdx.y;
 
-#ifdef MLA_TRACE
-    if (threadIdx.x == 0) {
-        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;
-        if (cta_ < 1024)
-            for (int e = 0; e < 16; ++e) g_ctatrace[cta_][e] = 0;
-        MLA_CTA_EVENT(0);
-    }
-    if (blockIdx.x < 2 && blockIdx.y == 0)
-        for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x)
-            (&g_trace[blockIdx.x][0][0])[i] = 0;
-#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
-            // bf16: one arrival + the pair's TMA bytes per piece; e4m3: the leader's widening warp
-            // arrives, the peer's signals by st.async
-            for (int j = 0; j < kKOps; ++j) mbar_init(bar(kBarKFull + kKOps * s + j), 1);
+            // bf16: one arrival + the pair's TMA bytes; e4m3: the leader's widening warp
+            // arrives, the peer's signal by st.async
+            mbar_init(bar(kBarKFull + s), 1);
             mbar_init(bar(kBarKEmpty + s), 1);
             mbar_init(bar(kBarQKDone + s), 1);
-            mbar_init(bar(kBarVFull + s), (kVTma && !kFp8) ? 1 : 4);
+            mbar_init(bar(kBarVFull + s), kFp8 ? 4 : 1);
             mbar_init(bar(kBarKRaw + s), 1);
         }
         // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
-        mbar_init(bar(kBarQFull), (kFp8 ? 0 : 1) + (kSignalAll ? 4 : 8));
+        mbar_init(bar(kBarQFull), (kFp8 ? 0 : 1) + 4);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
-            mbar_init(bar(kBarSFree + j), kSignalAll ? 4 : 8);
+            mbar_init(bar(kBarSFree + j), 4);
         }
-        mbar_init(bar(kBarPFull), kPSignalOnce ? 5 : (kPSignalAsync ? 4 : 8));
-        mbar_init(bar(kBarPLocal), 4);
+        mbar_init(bar(kBarPFull), 4);
         mbar_init(bar(kBarPvDone), 1);
         mbar_init(bar(kBarOFull), 1);
-        mbar_init(bar(kBarOEmpty), kSignalAll ? 4 : 8);
+        mbar_init(bar(kBarOEmpty), 4);
         mbar_init(bar(kBarXchg), 128);
         mbar_init(bar(kBarXchg + 1), 128);
         mbar_init(bar(kBarLx), 128);
@@ -405,26 +313,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     bool md_ok = true;
     UnitIter iter = make_iter(p, part, md_ok);
-    const uint64_t kv_pol = MLA_KV_EVICT_FIRST ? l2_policy_evict_first() : l2_policy_evict_normal();
+    const uint64_t kv_pol = l2_policy_evict_first();
     const uint64_t part_pol = l2_policy_evict_last();
     if (!md_ok && threadIdx.x == 0) raise_error(8 /* MLA_DEVERR_BAD_METADATA */);
 
-    // Signals to the leader's barriers: the leader's own warps arrive locally; the peer's
-    // warps arrive remotely, releasing at cluster scope only when they publish data.
-    auto arrive_leader = [&](int b_idx) {
-        __syncwarp();
-        if (lane == 0) {
-            if (leader)
-                mbar_arrive(bar(b_idx));
-            else
-                mbar_arrive_remote(map_to_cta(bar(b_idx), 0));
-        }
-    };
     // A warp publishing shared-memory data (written with st.shared, then fence.proxy.async by
-    // every writing thread) to the leader's MMA: the leader's warp arrives with expect_tx of 4
-    // bytes, the peer's warp sends a 4-byte st.async whose complete_tx lands on the leader's
-    // barrier (word: a landing slot of its own in the leader).  A remote release arrive took
-    // ~1000 cycles longer to reach the leader.
+    // every writing thread) or reporting a finished tensor-memory access to the leader's MMA
+    // issuer: the leader's warp arrives with expect_tx of 4 bytes, the peer's warp sends a
+    // 4-byte st.async whose complete_tx lands on the leader's barrier (word: a landing slot of
+    // its own in the leader).  A remote release arrive took ~1000 cycles longer to reach the
+    // leader.
     auto signal_leader = [&](int b_idx, int word) {
         __syncwarp();
         if (lane == 0) {
@@ -435,127 +333,47 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                              map_to_cta(bar(b_idx), 0));
         }
     };
-    auto arrive_leader_done_reading = [&](int b_idx) {
-        __syncwarp();
-        if (lane == 0) {
-            if (leader)
-                mbar_arrive(bar(b_idx));
-            else
-                mbar_arrive_remote_relaxed(map_to_cta(bar(b_idx), 0));
-        }
-    };
 
-    if (warp == 0 || warp == 2 || warp == 3) {
+    if (warp == 0 || warp == 3) {
         // ------------------------------------------------------------ K producers
         // Each tile's page (this CTA's page, all 576 columns) is one load, warps 0 / 3 taking
         // alternate tiles: 72 KB of bf16 completing the leader's barrier, or 36 KB of e4m3 that
-        // the loading warp widens in place before it signals the leader.  (Built with
-        // MLA_KOPS=3, the bf16 page comes in three 24 KB pieces by warps 0, 2 and 3, each on its
-        // own barrier, so that the S MMAs start on the first piece.)
-        constexpr bool alternate = kFp8 || kKOps == 1;   // one load per tile: warps 0 / 3 alternate
-        const int piece = alternate ? 0 : (warp == 0 ? 0 : (warp == 2 ? 1 : 2));
+        // the loading warp widens in place before it signals the leader.
         const uint32_t mine = warp == 3 ? 1u : 0u;
         uint32_t g = 0;
-        bool alive = !(alternate && warp == 2);
-#ifdef MLA_TRACE
-        if (alternate && warp == 2 && leader && lane == 0 && blockIdx.x < 2 && blockIdx.y == 0) {
-            // observer: completion time of each traced tile's barriers (leader CTA)
-            uint32_t total = 0;
-            {
-                UnitIter pk = iter;
-                int a, b0, b1;
-                while (pk.next(a, b0, b1)) total += (uint32_t)max(tiles_of(b0, b1), 0);
-            }
-            if (total > (uint32_t)kTraceTiles) total = kTraceTiles;
-            uint32_t gk = 0, gq = 0, gs = 0, gp = 0, gv = 0, gd = 0;
-            const long long t_start = clock64();
-            while (gd < total && clock64() - t_start < 400000000ll && !*abort_flag) {
-                if (gk < total && mbar_test_wait(bar(kBarKFull + kKOps * (gk & 1u)), (gk >> 1) & 1u))
-                    g_trace[0][gk++][24] = clock64();
-                if (gq < total && mbar_test_wait(bar(kBarQKDone + (gq & 1u)), (gq >> 1) & 1u))
-                    g_trace[0][gq++][25] = clock64();
-                if (gs < total && mbar_test_wait(bar(kBarSFull + (gs & 1u)), (gs >> 1) & 1u))
-                    g_trace[0][gs++][26] = clock64();
-                if (gp < total && mbar_test_wait(bar(kBarPFull), gp & 1u)) g_trace[0][gp++][27] = clock64();
-                if (gv < total && mbar_test_wait(bar(kBarVFull + (gv & 1u)), (gv >> 1) & 1u))
-                    g_trace[0][gv++][28] = clock64();
-                if (gd < total && mbar_test_wait(bar(kBarPvDone), gd & 1u)) g_trace[0][gd++][29] = clock64();
-            }
-        }
-#endif
+        bool alive = true;
         int ub, kb0, kb1;
         while (alive && iter.next(ub, kb0, kb1)) {
             const int n = tiles_of(kb0, kb1);
             if (n <= 0) continue;
             PageWindow pw;
             pw.init(p.block_table + (int64_t)ub * p.bt_stride, kb0, kb1, lane, p.num_pages, warp == 0);
-            int nx_ub = -1, nx_kb0 = 0, nx_kb1 = 0;   // the next unit with tiles, for the prefetch
-            {
-                UnitIter pk = iter;
-                int a, b0, b1;
-                while (pk.next(a, b0, b1)) {
-                    if (tiles_of(b0, b1) > 0) {
-                        nx_ub = a;
-                        nx_kb0 = b0;
-                        nx_kb1 = b1;
-                        break;
-                    }
-                }
-            }
             for (int i = 0; i < n; ++i, ++g) {
                 const int32_t row = pw.row(kb0 + 2 * i + (int)rank);
-                if (alternate && (g & 1u) != mine) continue;
+                if ((g & 1u) != mine) continue;
                 int ok = 1;
                 const int s = (int)(g & 1u);
                 const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                 if (lane == 0) {
-                    ok = mbar_wait_bounded<false>(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, abort_flag);
+                    ok = mbar_wait_bounded(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, abort_flag);
                     if (ok) {
                         if constexpr (kFp8) {
                             mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
-                            if (kL2Hints)
-                                tma_load_3d_hint(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0, kv_pol);
-                            else
-                                tma_load_3d(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0);
+                            tma_load_3d_hint(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0, kv_pol);
                         } else {
-                            const uint32_t kf = bar(kBarKFull + kKOps * s + piece);
-                            if (leader) mbar_arrive_expect_tx(kf, 2 * kKOpChunks * kBox);
-                            if (kL2Hints)
-                                tma_load_3d_pair_hint(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0,
-                                                      row, piece * kKOpChunks, kv_pol);
-                            else
-                                tma_load_3d_pair(slot + piece * kKOpChunks * kBox, &k_map, map_to_cta(kf, 0), 0, row,
-                                                 piece * kKOpChunks);
+                            const uint32_t kf = bar(kBarKFull + s);
+                            if (leader) mbar_arrive_expect_tx(kf, 2 * kChunks * kBox);
+                            tma_load_3d_pair_hint(slot, &k_map, map_to_cta(kf, 0), 0, row, 0, kv_pol);
                         }
-                        if (piece == 0) MLA_TRACE_EVENT(g, 12);
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     alive = false;
                     break;
                 }
-                if constexpr (kL2Prefetch) {
-                    // this warp's next tile: two tiles on, possibly in the part's next unit
-                    int ti = i + 2, tkb0 = kb0, tkb1 = kb1, tub = ub;
-                    if (ti >= n) {
-                        ti -= n;
-                        tkb0 = nx_kb0;
-                        tkb1 = nx_kb1;
-                        tub = nx_ub;
-                    }
-                    const int blk_next = tkb0 + 2 * ti + (int)rank;
-                    if (alternate && tub >= 0 && blk_next < tkb1) {
-                        const int pn = __ldg(p.block_table + (int64_t)tub * p.bt_stride + blk_next);
-                        if (pn >= 0 && (int64_t)pn < p.num_pages) {
-                            constexpr int kRowBytes = kFp8 ? kDqk : 2 * kDqk;
-                            const uint8_t* base = p.kv + (int64_t)pn * kPage * kRowBytes;
-                            for (int l = lane; l < kPage * kRowBytes / 128; l += 32) prefetch_l2(base + 128 * l);
-                        }
-                    }
-                }
                 if constexpr (kFp8) {
                     // the whole warp widens the page in place, then signals the leader
-                    const bool landed = mbar_wait_bounded<false>(bar(kBarKRaw + s), (g >> 1) & 1u, abort_flag);
+                    const bool landed = mbar_wait_bounded(bar(kBarKRaw + s), (g >> 1) & 1u, abort_flag);
                     if (!__all_sync(0xffffffffu, landed)) {
                         alive = false;
                         break;
@@ -564,7 +382,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     for (int c = 0; c < kChunks; ++c)
                         widen_chunk_e4m3(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
                     fence_proxy_async_smem();
-                    signal_leader(kBarKFull + kKOps * s, 8);
+                    signal_leader(kBarKFull + s, 8);
                 }
             }
         }
@@ -613,7 +431,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             const int n = tiles_of(kb0, kb1);
             if (n <= 0) continue;
             // ---- Q of the unit
-            if (uq > 0 && !mbar_wait_bounded<false>(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
+            if (uq > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
             tc_fence_after();
             if (!kFp8 && quarter == 3 && lane == 0) {
                 if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQHiBytes);
@@ -663,10 +481,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             }
             tc_wait_st();
             tc_fence_before();
-            if (kSignalAll)
-                signal_leader(kBarQFull, 9 + quarter);
-            else
-                arrive_leader(kBarQFull);
+            signal_leader(kBarQFull, 9 + quarter);
             ++uq;
             // ---- partner V of each tile of the unit
             const int32_t* bt_row = p.block_table + (int64_t)ub * p.bt_stride;
@@ -676,25 +491,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (pg < 0 || (int64_t)pg >= p.num_pages) pg = -1;   // reported by the K loads
                 const int s = (int)(g & 1u);
                 const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
-                if constexpr (kVTma && !kFp8) {
+                if constexpr (!kFp8) {
                     // by TMA, after the tile's S MMAs: two 16 KB loads, lane 0 of the last warp
                     if (quarter == 3) {
                         int ok = 1;
                         if (lane == 0) {
-                            ok = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                            ok = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
                             if (ok) {
                                 if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * 2 * 2 * kBox);
                                 const int32_t row = pg >= 0 ? pg * kPage : (int32_t)(p.num_pages * kPage);
 #pragma unroll
                                 for (int nn = 0; nn < 2; ++nn)
-                                    if (kL2Hints)
-                                        tma_load_3d_pair_hint(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
-                                                              map_to_cta(bar(kBarVFull + s), 0), 0, row,
-                                                              4 * nn + 2 * (int)rank, kv_pol);
-                                    else
-                                        tma_load_3d_pair(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
-                                                         map_to_cta(bar(kBarVFull + s), 0), 0, row, 4 * nn + 2 * (int)rank);
-                                MLA_TRACE_EVENT(g, 18);
+                                    tma_load_3d_pair_hint(slot + (4 * nn + 2 * (1 - (int)rank)) * kBox, &v_map,
+                                                          map_to_cta(bar(kBarVFull + s), 0), 0, row,
+                                                          4 * nn + 2 * (int)rank, kv_pol);
                             }
                         }
                         if (!__shfl_sync(0xffffffffu, ok, 0)) {
@@ -702,10 +512,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                             break;
                         }
                     }
-                    continue;
-                }
-                if constexpr (kFp8) {
-                    // 4 chunks x 64 rows x 4 sixteen-byte units of e4m3: 8 per thread
+                } else {
+                    // 4 chunks x 64 rows x 4 sixteen-byte units of e4m3: 8 per thread, widened to
+                    // f16 on the way into the slot
                     uint4 v[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -715,7 +524,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                              p.kv + ((int64_t)pg * kPage + row) * kDqk + chunk * 64 + q4 * 16))
                                        : make_uint4(0, 0, 0, 0);
                     }
-                    const bool done = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                    const bool done = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
                     if (!__all_sync(0xffffffffu, done)) {
                         alive = false;
                         break;
@@ -732,35 +541,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                       e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w),
                                       e4m3x2_to_f16x2(v[j].w >> 16));
                     }
-                } else {
-                    // 4 chunks x 64 rows x 8 sixteen-byte units of bf16: 16 per thread
-                    uint4 v[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int x = qt + 128 * j, h = x >> 9, row = (x >> 3) & 63, u = x & 7;
-                        const int chunk = 4 * (h >> 1) + 2 * (int)rank + (h & 1);
-                        v[j] = pg >= 0 ? __ldg(reinterpret_cast<const uint4*>(
-                                             p.kv + ((int64_t)pg * kPage + row) * (2 * kDqk) + chunk * 128 + u * 16))
-                                       : make_uint4(0, 0, 0, 0);
-                    }
-                    if (qt == 0) MLA_TRACE_EVENT(g, 19);
-                    const bool done = mbar_wait_bounded<false>(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
-                    if (!__all_sync(0xffffffffu, done)) {
-                        alive = false;
-                        break;
-                    }
-                    if (qt == 0) MLA_TRACE_EVENT(g, 20);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int x = qt + 128 * j, h = x >> 9, row = (x >> 3) & 63, u = x & 7;
-                        const int pos = 4 * (h >> 1) + 2 * (1 - (int)rank) + (h & 1);
-                        st_shared_v4u(slot + pos * kBox + row * 128 + 16u * ((uint32_t)u ^ ((uint32_t)row & 7u)),
-                                      v[j].x, v[j].y, v[j].z, v[j].w);
-                    }
+                    fence_proxy_async_smem();
+                    signal_leader(kBarVFull + s, 4 + quarter);
                 }
-                if (qt == 0) MLA_TRACE_EVENT(g, 18);
-                fence_proxy_async_smem();
-                signal_leader(kBarVFull + s, 4 + quarter);
             }
         }
         if (!kFp8 && quarter == 3 && lane == 0 && *abort_flag) {
@@ -778,13 +561,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // unit, the unit's Q; PV(t) waits for P(t), the partner V of tile t and, first in a
         // unit, the epilogue of the previous unit having read O.
         if (leader && lane == 0) {
-            // non-blocking barrier test for the polling loop
-            auto poll = [](uint32_t b, uint32_t parity) -> bool {
-                return kIssuerPollCta ? mbar_test_wait(b, parity) : mbar_test_wait_cluster(b, parity);
-            };
+            // Non-blocking barrier tests at CTA scope: the data behind a barrier the peer
+            // completes is ordered by the peer's fence.proxy.async and the st.async / TMA
+            // complete_tx itself (measured ~1% faster than cluster-scope acquire).
+            auto poll = [](uint32_t b, uint32_t parity) -> bool { return mbar_test_wait(b, parity); };
             struct Cursor {
                 UnitIter it;
-                int n, i, piece;
+                int n, i;
                 uint32_t g, uq;
                 bool valid;
                 __device__ void next_unit() {
@@ -801,7 +584,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 __device__ void step() {
                     ++g;
-                    piece = 0;
                     if (++i == n) {
                         ++uq;
                         next_unit();
@@ -812,37 +594,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             cq.it = iter;
             cq.g = 0;
             cq.uq = 0;
-            cq.piece = 0;
             cq.next_unit();
             cp = cq;
             uint64_t t_idle = global_timer_ns();
-#ifdef MLA_TRACE
-            uint32_t tr_g = 0xffffffffu;
-            bool tr_p = false, tr_v = false;
-#endif
             while (cq.valid || cp.valid) {
                 bool did = false;
                 if (cp.valid && cp.g < cq.g) {
                     const int s = (int)(cp.g & 1u);
                     const bool first = cp.i == 0;
-#ifdef MLA_TRACE
-                    if (tr_g != cp.g) {
-                        tr_g = cp.g;
-                        tr_p = tr_v = false;
-                    }
-                    if (!tr_p && poll(bar(kBarPFull), cp.g & 1u)) {
-                        tr_p = true;
-                        MLA_TRACE_EVENT(cp.g, 21);
-                    }
-                    if (!tr_v && poll(bar(kBarVFull + s), (cp.g >> 1) & 1u)) {
-                        tr_v = true;
-                        MLA_TRACE_EVENT(cp.g, 22);
-                    }
-#endif
                     if (poll(bar(kBarPFull), cp.g & 1u) && poll(bar(kBarVFull + s), (cp.g >> 1) & 1u) &&
                         (!first || cp.uq == 0 || poll(bar(kBarOEmpty), (cp.uq - 1) & 1u))) {
                         tc_fence_after();
-                        MLA_TRACE_EVENT(cp.g, 2);
                         const uint32_t pbuf = sbase + kOffP;
                         const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
 #pragma unroll
@@ -858,27 +620,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_commit_pair(bar(kBarKEmpty + s));
                         tc_commit_pair(bar(kBarPvDone));
                         if (cp.i == cp.n - 1) tc_commit_pair(bar(kBarOFull));
-                        MLA_TRACE_EVENT(cp.g, 14);
                         cp.step();
                         did = true;
                     }
                 }
                 if (!did && cq.valid) {
-                    // S in the pieces the page arrives in (one, unless built with MLA_KOPS=3)
                     const int s = (int)(cq.g & 1u);
                     const uint32_t sb = cq.g & 1u;
-                    const int j = cq.piece;
-                    if ((j != 0 || cq.i != 0 || poll(bar(kBarQFull), cq.uq & 1u)) &&
-                        (j != 0 || cq.g < 2 || poll(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
-                        poll(bar(kBarKFull + kKOps * s + (kFp8 ? 0 : j)), (cq.g >> 1) & 1u)) {
+                    if ((cq.i != 0 || poll(bar(kBarQFull), cq.uq & 1u)) &&
+                        (cq.g < 2 || poll(bar(kBarSFree + sb), ((cq.g >> 1) & 1u) ^ 1u)) &&
+                        poll(bar(kBarKFull + s), (cq.g >> 1) & 1u)) {
                         tc_fence_after();
-                        MLA_TRACE_EVENT(cq.g, 15 + j);
-                        if (j == 0 && cq.i == 0 && cq.uq < 6) MLA_CTA_EVENT(3 + 2 * cq.uq);
                         const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                         const uint32_t d = tmem + kTmemS + 64u * sb;
 #pragma unroll
-                        for (int cc = 0; cc < kKOpChunks; ++cc) {
-                            const int c = kKOpChunks * j + cc;
+                        for (int c = 0; c < kChunks; ++c) {
                             if (c < kQLoChunks) {
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
@@ -893,15 +649,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                                 kFp8 ? kIdescQK16 : kIdescQK, 1u);
                             }
                         }
-                        if (j == kKOps - 1) {
-                            tc_commit_pair(bar(kBarQKDone + s));
-                            tc_commit_pair(bar(kBarSFull + sb));
-                            if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
-                            MLA_TRACE_EVENT(cq.g, 13);
-                            cq.step();
-                        } else {
-                            ++cq.piece;
-                        }
+                        tc_commit_pair(bar(kBarQKDone + s));
+                        tc_commit_pair(bar(kBarSFull + sb));
+                        if (cq.i == cq.n - 1) tc_commit_pair(bar(kBarQEmpty));
+                        cq.step();
                         did = true;
                     }
                 }
@@ -960,12 +711,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             float m_run = -INFINITY, l_half = 0.f;
             for (int i = 0; i < n; ++i, ++g) {
                 const uint32_t sb = g & 1u;
-                if (t == 0) MLA_TRACE_EVENT(g, 3);
-                if (!mbar_wait_bounded<false>(bar(kBarSFull + sb), (g >> 1) & 1u, abort_flag)) {
+                if (!mbar_wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, abort_flag)) {
                     alive = false;
                     break;
                 }
-                if (t == 0) MLA_TRACE_EVENT(g, 4);
                 tc_fence_after();
                 float s[64];
                 {
@@ -979,13 +728,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 #pragma unroll
                         for (int k = 0; k < 16; ++k) s[16 * c + k] = __uint_as_float(raw[c][k]);
                 }
-                if (t == 0) MLA_TRACE_EVENT(g, 11);
                 tc_fence_before();
-                if (kSignalAll)
-                    signal_leader(kBarSFree + sb, 16 + (warp - kSoftmaxWarp0));
-                else
-                    arrive_leader_done_reading(kBarSFree + sb);
-                if (t == 0) MLA_TRACE_EVENT(g, 7);
+                signal_leader(kBarSFree + sb, 16 + (warp - kSoftmaxWarp0));
                 // scale to log2 units, mask, this half's maximum
                 const int kbase = (kb0 + 2 * i) * kPage + kPage * half;
                 float hmax = -INFINITY;
@@ -998,13 +742,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 // partner thread t ^ 64 holds the other 64 tokens of this row
                 xmax[sb * 128 + t] = hmax;
-                if (t == 0) MLA_TRACE_EVENT(g, 8);
                 mbar_arrive(bar(kBarXchg + sb));
-                if (!mbar_wait_bounded<false>(bar(kBarXchg + sb), (g >> 1) & 1u, abort_flag)) {
+                if (!mbar_wait_bounded(bar(kBarXchg + sb), (g >> 1) & 1u, abort_flag)) {
                     alive = false;
                     break;
                 }
-                if (t == 0) MLA_TRACE_EVENT(g, 9);
                 const float tmax = fmaxf(hmax, xmax[sb * 128 + (t ^ 64)]);
                 const float m_new = fmaxf(m_run, tmax);
                 const bool rescale = m_new > m_run + kRescaleThreshold;
@@ -1026,11 +768,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     s[j] = __uint_as_float(kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1));
                 }
                 l_half += psum;
-                if (t == 0) MLA_TRACE_EVENT(g, 5);
                 // the P buffer is free, and O holds every PV up to tile g - 1, once PV(g - 1)
                 // has finished
-                if (t == 0) MLA_TRACE_EVENT(g, 10);
-                if (g >= 1 && !mbar_wait_bounded<false>(bar(kBarPvDone), (g - 1) & 1u, abort_flag)) {
+                if (g >= 1 && !mbar_wait_bounded(bar(kBarPvDone), (g - 1) & 1u, abort_flag)) {
                     alive = false;
                     break;
                 }
@@ -1060,35 +800,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                       __float_as_uint(s[4 * c + 3]));
                 }
                 fence_proxy_async_smem();
-                if (t == 0) MLA_TRACE_EVENT(g, 23);
-                if (kPSignalAsync) {
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (leader)
-                            mbar_arrive_expect_tx(bar(kBarPFull), 4);
-                        else
-                            st_async_b32(map_to_cta(sbase + kOffPSig + 4u * (uint32_t)(warp - kSoftmaxWarp0), 0), g,
-                                         map_to_cta(bar(kBarPFull), 0));
-                    }
-                } else if (kPSignalOnce && !leader) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(kBarPLocal));
-                    if (t == 0) {
-                        if (mbar_wait_bounded<false>(bar(kBarPLocal), g & 1u, abort_flag))
-                            mbar_arrive_remote(map_to_cta(bar(kBarPFull), 0));
-                    }
-                } else {
-                    arrive_leader(kBarPFull);
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive_expect_tx(bar(kBarPFull), 4);
+                    else
+                        st_async_b32(map_to_cta(sbase + kOffPSig + 4u * (uint32_t)(warp - kSoftmaxWarp0), 0), g,
+                                     map_to_cta(bar(kBarPFull), 0));
                 }
-                if (t == 0) MLA_TRACE_EVENT(g, 6);
             }
             if (!alive) break;
             // epilogue of the unit
-            if (!mbar_wait_bounded<false>(bar(kBarOFull), uq & 1u, abort_flag)) break;
+            if (!mbar_wait_bounded(bar(kBarOFull), uq & 1u, abort_flag)) break;
             tc_fence_after();
             xmax[256 + t] = l_half;
             mbar_arrive(bar(kBarLx));
-            if (!mbar_wait_bounded<false>(bar(kBarLx), uq & 1u, abort_flag)) break;
+            if (!mbar_wait_bounded(bar(kBarLx), uq & 1u, abort_flag)) break;
             const float l_run = l_half + xmax[256 + (t ^ 64)];
             const int pieces = p.num_splits[ub + 1] - p.num_splits[ub];
             const bool direct = pieces == 1;
@@ -1118,10 +845,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_wait_ld();
                         if (st == steps - 1) {
                             tc_fence_before();
-                            if (kSignalAll)   // O is free for the next unit
-                                signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));
-                            else
-                                arrive_leader_done_reading(kBarOEmpty);
+                            signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));   // O is free for the next unit
                         }
 #pragma unroll
                         for (int k = 0; k < 32; ++k)
@@ -1135,10 +859,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_wait_ld();
                         if (st == steps - 1) {
                             tc_fence_before();
-                            if (kSignalAll)   // O is free for the next unit
-                                signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));
-                            else
-                                arrive_leader_done_reading(kBarOEmpty);
+                            signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));   // O is free for the next unit
                         }
 #pragma unroll
                         for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * inv);
@@ -1159,23 +880,18 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         if (rg < p.rows) {
                             if (direct)
                                 *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
-                            else if (kL2Hints)
-                                st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
                             else
-                                *reinterpret_cast<uint4*>(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u) = v;
+                                st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
                         }
                     }
                     __syncwarp();
                 }
             }
-            if (t == 0 && uq < 6) MLA_CTA_EVENT(4 + 2 * uq);
             if (row_valid && half == 0) {
                 if (direct)
                     p.lse[(int64_t)ub * p.rows + rowg] = lse_val;
-                else if (kL2Hints)
-                    st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
                 else
-                    p.part_lse[(int64_t)split * p.rows + rowg] = lse_val;
+                    st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
             }
             ++uq;
         }
@@ -1183,7 +899,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) MLA_CTA_EVENT(2);
     cluster_sync();
     if (warp == 1) {
         tc_fence_after();

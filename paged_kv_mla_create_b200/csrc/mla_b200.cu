@@ -82,7 +82,7 @@ const char* mla_status_string(mla_status_t s) {
     return "MLA_ERR_UNKNOWN";
 }
 
-int32_t mla_abi_version(void) { return 1; }
+int32_t mla_abi_version(void) { return 2; }
 
 mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t req_to_token_rows,
                                    int64_t req_to_token_stride, const void* req_pool_indices,
@@ -122,10 +122,12 @@ int32_t mla_num_sm_parts(int32_t sm_count, int32_t num_heads_per_head_k, int32_t
 }
 
 mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
-                                  int32_t num_sm_parts, int32_t is_fp8_kvcache,
+                                  int32_t num_heads_per_head_k, int32_t num_heads_k,
+                                  int32_t is_fp8_kvcache, int32_t sm_count,
                                   int32_t* tile_scheduler_metadata, int32_t* num_splits,
                                   mla_stream_t stream) {
     (void)is_fp8_kvcache;  // accepted for call compatibility; the plan does not depend on it
+    const int32_t num_sm_parts = mla_num_sm_parts(sm_count, num_heads_per_head_k, num_heads_k);
     if (bs < 0 || num_sm_parts < 1 || bs > (1 << 20)) return MLA_ERR_INVALID_ARG;
     if (!tile_scheduler_metadata || !num_splits || (bs > 0 && !cache_seqlens))
         return MLA_ERR_INVALID_ARG;
@@ -157,6 +159,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     if (head_dim != 576 || head_dim_v != 512 || page_size != 64) return MLA_ERR_UNSUPPORTED;
     if (q_dtype != MLA_DTYPE_BF16) return MLA_ERR_UNSUPPORTED;
     if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+    if (kv_dtype == MLA_DTYPE_BF16 && descale_k) return MLA_ERR_INVALID_ARG;  // fp8 caches only
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (bs == 0) return MLA_OK;
@@ -165,7 +168,8 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
         return MLA_ERR_INVALID_ARG;
     if (num_pages <= 0 || num_pages * 64 >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
     if (max_pages <= 0 || block_table_stride < max_pages) return MLA_ERR_INVALID_ARG;
-    if ((int64_t)q_len * h_q > (int64_t(1) << 24) || bs > 65535) return MLA_ERR_UNSUPPORTED;
+    // grid.y = cdiv(q_len * h_q, 128) query tiles, at most 65535
+    if ((int64_t)q_len * h_q > int64_t(65535) * 128 || bs > 65535) return MLA_ERR_UNSUPPORTED;
     if (!is_aligned(q, 16) || !is_aligned(k_cache, 16) || !is_aligned(out, 16) ||
         !is_aligned(tile_scheduler_metadata, 16))
         return MLA_ERR_INVALID_ARG;
@@ -181,7 +185,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // view orders its dimensions so that one load lands as consecutive 64-row x 64-column
     // boxes (8 KB each), the layout the MMAs read:
     //   K: (64 columns, pool rows [1152 B], 9 column chunks [128 B]); a load = all nine
-    //      column chunks of one page (72 KB; three chunks, 24 KB, when built with MLA_KOPS=3).
+    //      column chunks of one page (72 KB).
     //   V: the same view with a box of two column chunks (16 KB): a partner page's V chunks.
     //   Q: (64 columns, rows of a request [1152 B], 9 column chunks [128 B], requests); a load
     //      = 64 query rows x columns [256, 576) (40 KB).
@@ -195,7 +199,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     if (!fp8) {
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {1152, 128};
-        const cuuint32_t kbox[3] = {64, 64, (cuuint32_t)mla::decode::kKOpChunks};
+        const cuuint32_t kbox[3] = {64, 64, (cuuint32_t)mla::decode::kChunks};
         const cuuint32_t vbox[3] = {64, 64, 2};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), gdim, gstride,
@@ -339,15 +343,3 @@ extern "C" mla_status_t mla_decode_paged_noalloc(
                             softmax_scale, causal, descale_q, descale_k, out, lse, scratch,
                             MLA_NOALLOC_SCRATCH_BYTES, stream);
 }
-
-#ifdef MLA_TRACE
-// Trace builds only: copy the pipeline trace to the host.
-extern "C" __attribute__((visibility("default"))) int mla_trace_dump(void* host, size_t bytes) {
-    if (bytes > sizeof(mla::decode::g_trace)) bytes = sizeof(mla::decode::g_trace);
-    return (int)cudaMemcpyFromSymbol(host, mla::decode::g_trace, bytes);
-}
-extern "C" __attribute__((visibility("default"))) int mla_ctatrace_dump(void* host, size_t bytes) {
-    if (bytes > sizeof(mla::decode::g_ctatrace)) bytes = sizeof(mla::decode::g_ctatrace);
-    return (int)cudaMemcpyFromSymbol(host, mla::decode::g_ctatrace, bytes);
-}
-#endif

@@ -42,31 +42,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// Arrive on an mbarrier in a peer CTA's shared memory (cluster address from mapa),
-// releasing this thread's prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-                 : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Acquire at cluster scope: pairs with mbar_arrive_remote from the peer CTA.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -88,33 +68,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Wait budget for one pipeline wait.  Every wait in the kernels is bounded: after this
 // many nanoseconds without the phase completing the waiter records
 // MLA_DEVERR_WAIT_TIMEOUT, raises the CTA's abort flag and returns false; a raised abort
 // flag makes every later wait return false at once so that all roles drain to the exit.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
-template <bool kCluster>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag) {
-    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (*abort_flag) return false;
-        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity))
-            return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if (global_timer_ns() - t0 > kWaitBudgetNs) {
             raise_error(16 /* MLA_DEVERR_WAIT_TIMEOUT */);
             *abort_flag = 1;
@@ -152,11 +118,6 @@ __device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// Hint the L2 to fetch the 128-byte line holding addr (no data returns to the SM).
-__device__ __forceinline__ void prefetch_l2(const void* addr) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
@@ -219,27 +180,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // ------------------------------------------------------------------ pair (cta_group::2)
-// TMA load into this CTA's shared memory, completing on this CTA's mbarrier.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t c0, int32_t c1, int32_t c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// TMA load whose bytes complete on an mbarrier of the pair's leader CTA (cluster address).
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map,
-                                                 uint32_t leader_bar, int32_t c0, int32_t c1,
-                                                 int32_t c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map,
                                                  uint32_t leader_bar, int32_t c0, int32_t c1,
                                                  int32_t c2, int32_t c3) {
@@ -251,19 +191,11 @@ __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap
 }
 
 // ------------------------------------------------------------------ L2 eviction priority
-#ifndef MLA_L2_HINTS
-#define MLA_L2_HINTS 1
-#endif
 // Cache policies (createpolicy, applied to the whole access): the KV stream is read once and
 // goes first; the split partials are read back by the merge right after and should stay.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
@@ -272,7 +204,8 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     return pol;
 }
 
-// As tma_load_3d / tma_load_3d_pair with an L2 cache policy.
+// 3-D TMA loads with an L2 cache policy: into this CTA's shared memory completing on its own
+// mbarrier, or (pair) completing on an mbarrier of the pair's leader CTA (cluster address).
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                                  int32_t c0, int32_t c1, int32_t c2, uint64_t pol) {
     asm volatile(
@@ -321,13 +254,6 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t 
     asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
                  "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-
-// Arrive on a peer CTA's mbarrier without ordering this thread's memory accesses (for
-// signals whose data dependence was already resolved, e.g. a completed tensor-memory read).
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
                  : "memory");
 }
 

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = mla.library()
-    assert lib.mla_abi_version() == 1
+    assert lib.mla_abi_version() == 2
     for code, name in mla._STATUS.items():
         assert lib.mla_status_string(code).decode() == name
 
@@ -84,6 +84,8 @@ def test_decode_validation_happens_before_any_launch():
     assert _decode(lib, ws_bytes=16) == 5                # workspace too small
     assert _decode(lib, ws=None) == 5
     assert _decode(lib, scale=float("nan")) == 1
+    assert _decode(lib, dk=1 << 29) == 1                 # descale_k with a bf16 cache
+    assert _decode(lib, q_len=1, h_q=65535 * 128 + 1) == 2   # more query tiles than grid.y holds
 
 
 def test_block_table_and_planner_validation():
@@ -97,6 +99,10 @@ def test_block_table_and_planner_validation():
     assert bt(*{**ok, "out_stride": 2}.values()) == 1
     assert bt(*{**ok, "r2t": None}.values()) == 1
     md = lib.mla_get_mla_metadata
-    assert md(1 << 20, 2, 0, 0, 1 << 21, 1 << 22, None) == 1
-    assert md(1 << 20, -1, 74, 0, 1 << 21, 1 << 22, None) == 1
-    assert md(1 << 20, 2, 74, 0, (1 << 21) + 4, 1 << 22, None) == 1   # misaligned rows
+    # (cache_seqlens, bs, num_heads_per_head_k, num_heads_k, is_fp8, sm_count, md, ns, stream)
+    assert md(1 << 20, 2, 0, 1, 0, 148, 1 << 21, 1 << 22, None) == 1     # no heads
+    assert md(1 << 20, 2, 128, 0, 0, 148, 1 << 21, 1 << 22, None) == 1   # no KV heads
+    assert md(1 << 20, 2, 128, 1, 0, 0, 1 << 21, 1 << 22, None) == 1     # no SMs
+    assert md(1 << 20, -1, 128, 1, 0, 148, 1 << 21, 1 << 22, None) == 1
+    assert md(1 << 20, 2, 128, 1, 0, 148, (1 << 21) + 4, 1 << 22, None) == 1   # misaligned rows
+    assert md(1 << 20, 2, 128, 1, 0, 148, None, 1 << 22, None) == 1

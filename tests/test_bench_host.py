@@ -22,17 +22,26 @@ def test_roofline_hbm_bound_decode():
 
 
 def test_roofline_fp8_cache_reports_both_peaks():
-    # e4m3 cache: half the KV bytes, the same FLOPs -> tensor-bound at the bf16 (f16 MMA) peak,
-    # also reported against the fp8 peak (2x)
+    # e4m3 cache: half the KV bytes, the same FLOPs -> bound by the fp8 tensor peak (the
+    # measured bf16 peak x 2), also reported against the bf16 peak its f16 MMAs run at
     kv, q, fl, t = 150e6, 18.9e6, 146e9, 256.6e-6
     r = bench.roofline_entry(kv, q, fl, t, PEAKS, "measured", True, None)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert math.isclose(r["achieved"], fl / t / 1e12)
-    assert math.isclose(r["frac"], r["achieved"] / PEAKS["bf16_tflops"])
-    assert math.isclose(r["fp8_peak_tflops"], 2 * PEAKS["bf16_tflops"])
-    assert math.isclose(r["frac_of_fp8_peak"], r["frac"] / 2)
+    assert math.isclose(r["peak"], 2 * PEAKS["bf16_tflops"])
+    assert math.isclose(r["frac"], r["achieved"] / (2 * PEAKS["bf16_tflops"]))
+    assert math.isclose(r["frac_of_bf16_peak"], 2 * r["frac"])
+    assert r["tensor_peak_dtype"] == "fp8"
     assert r["traffic"] is None
     json.dumps(r)
+
+
+def test_roofline_fp8_cache_can_be_hbm_bound():
+    # fewer FLOPs per byte: at the fp8 peak the HBM time is the slower one
+    kv, q, fl, t = 300e6, 18.9e6, 100e9, 100e-6
+    r = bench.roofline_entry(kv, q, fl, t, PEAKS, "measured", True, None)
+    assert r["bound"] == "hbm"
+    assert math.isclose(r["frac"], (kv + q) / t / 1e9 / PEAKS["hbm_gbs"])
 
 
 def test_roofline_fallback_peak_is_named():

@@ -181,14 +181,17 @@ def test_bad_page_id_is_reported_not_faulted(mla):
 
 # ------------------------------------------------------------------ full-size workloads
 def sample_rows(wl, n, seed):
+    """n random rows, plus, for every request and every query position, its first head, its
+    last head and one random head: every request, every draft position and both ends of the
+    head range are compared with the oracle."""
     rng = np.random.default_rng(seed)
     total = wl.bs * wl.q_len * wl.h
-    rows = rng.choice(total, size=min(n, total), replace=False)
-    # always include the longest request and both ends of the row range
-    b_long = int(np.argmax(wl.cache_seqlens.numpy()))
-    per = wl.q_len * wl.h
-    extra = [0, total - 1, b_long * per, b_long * per + per - 1]
-    return np.unique(np.concatenate([rows, extra])).astype(np.int64)
+    rows = [rng.choice(total, size=min(n, total), replace=False)]
+    for b in range(wl.bs):
+        for i in range(wl.q_len):
+            base = (b * wl.q_len + i) * wl.h
+            rows.append(np.array([base, base + wl.h - 1, base + int(rng.integers(0, wl.h))]))
+    return np.unique(np.concatenate(rows)).astype(np.int64)
 
 
 @pytest.mark.parametrize("index", [2, 3, 4, 5])
@@ -205,6 +208,99 @@ def test_full_size_workload_sampled(mla, index):
     # log of one allowed key's weight (lse > -inf) for every live row
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     assert mla.read_device_error() == 0
+
+
+# ------------------------------------------------------------------ degenerate and graph-mode cases
+@pytest.mark.parametrize("parts", [None, 7])
+def test_verify_rows_without_allowed_keys(mla, parts):
+    """Causal multi-query rows whose limit L - q_len + i + 1 is <= 0 (a cache shorter than the
+    draft) see no key: o = 0 and lse = -inf, as the oracle pins; the others see a prefix."""
+    wl = W.make_case([2, 1, 3, 0, 100, 5, 700], h=128, q_len=4, verify=False, seed=41, poison=True)
+    assert wl.causal and wl.num_draft_tokens == 0
+    check_full(mla, wl, parts)
+
+
+def _plan_with_lone_last_block(q_len):
+    """A single request of L = 64k + 2 keys and a part count whose plan makes the request's
+    final piece its last block alone: that piece holds only keys past the causal limit of
+    draft rows i < q_len - 2, so those rows' partial state there is empty (lse = -inf)."""
+    for k in range(2, 60):
+        L = 64 * k + 2
+        for parts in range(2, 40):
+            md, ns = oracle.get_mla_metadata(np.array([L], dtype=np.int32), parts)
+            if ns[1] < 2:
+                continue
+            last = [r for r in md if r[0] == 0 and r[2] == 1 and r[1] == k]   # piece [k, k+1)
+            if last:
+                return L, parts
+    raise AssertionError("no plan with a one-block final piece")
+
+
+def test_wholly_masked_split_piece(mla):
+    L, parts = _plan_with_lone_last_block(4)
+    wl = W.make_case([L - 4], h=128, q_len=4, verify=True, seed=42, poison=True)
+    assert int(wl.cache_seqlens[0]) == L
+    md, ns = oracle.get_mla_metadata(wl.cache_seqlens, parts)
+    assert ns[1] >= 2
+    check_full(mla, wl, parts)
+
+
+def test_graph_mode_page_table(mla):
+    """The graph-capture branch: a [max_bs, stride] table pre-filled with 1, a request-pool
+    of 4096 rows, and fill_tail off: entries below cdiv(L, 64) match the oracle bit for bit,
+    every other entry (also the columns past max_pages) keeps its 1."""
+    wl = W.make_case([700, 65, 1, 0, 2049], h=16, seed=43)
+    rng = np.random.default_rng(43)
+    big_rows = rng.choice(4096, size=wl.bs, replace=False)
+    r2t = torch.zeros((4096, wl.req_to_token.shape[1]), dtype=torch.int32)
+    r2t[big_rows] = wl.req_to_token[wl.req_pool_indices]
+    rpi = torch.tensor(big_rows, dtype=torch.int64)
+    stride = wl.max_pages + 9
+    table = torch.ones((wl.bs + 3, stride), dtype=torch.int32, device="cuda")
+    out = table[:wl.bs, :wl.max_pages]
+    mla.build_block_table(r2t.cuda(), rpi.cuda(), wl.seq_lens.cuda(), wl.max_pages, out=out,
+                          fill_tail=False)
+    torch.cuda.synchronize()
+    got = table.cpu().numpy()
+    ref = oracle.build_block_table(r2t, rpi, wl.seq_lens, wl.max_pages)
+    npages = [-(-int(L) // 64) for L in wl.seq_lens]
+    for b in range(wl.bs):
+        assert np.array_equal(got[b, :npages[b]], ref[b, :npages[b]]), f"row {b}"
+        assert np.all(got[b, npages[b]:] == 1), f"row {b}: tail overwritten"
+    assert np.all(got[wl.bs:] == 1)
+    assert mla.read_device_error() == 0
+
+
+def test_misaligned_slots_are_reported(mla):
+    """req_to_token whose slots for one page do not start a page: the entry is still
+    slot / 64 (the oracle's value) and the error word records the broken precondition."""
+    wl = W.make_case([300, 130], h=16, seed=44)
+    r2t = wl.req_to_token.clone()
+    row = int(wl.req_pool_indices[0])
+    r2t[row, 64:128] += 1
+    bt = mla.build_block_table(r2t.cuda(), wl.req_pool_indices.cuda(), wl.seq_lens.cuda(),
+                               wl.max_pages)
+    torch.cuda.synchronize()
+    ref = oracle.build_block_table(r2t, wl.req_pool_indices, wl.seq_lens, wl.max_pages)
+    assert np.array_equal(bt.cpu().numpy(), ref)
+    assert mla.read_device_error() == 64
+    assert mla.read_device_error() == 0
+
+
+def test_q_out_of_f16_range_is_reported(mla):
+    """With an e4m3 cache the product runs in f16: a q value beyond 65504 (made on the host)
+    is recorded in the error word instead of silently overflowing."""
+    wl = W.make_case([200, 70], h=16, kv="fp8", seed=45)
+    wl.q[1, 0, 3, 17] = 70000.0
+    run_path(mla, wl)
+    assert mla.read_device_error() & 32
+
+
+def test_fp8_cache_tiny_q_values(mla):
+    """q values around 1e-6 (f16 subnormals in the e4m3 path) still meet the tolerance."""
+    wl = W.make_case([300, 1000, 65], h=128, kv="fp8", seed=46)
+    wl.q.mul_(1e-6)
+    check_full(mla, wl)
 
 
 # ------------------------------------------------------------------ planner, random batches
