@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the paged MLA decode hot path on B200.
 
-One step = one pass of the whole path over one batch: page table (build_block_table),
-split plan (get_mla_metadata) and attention with its split merge (mla_decode_paged),
+One step = one pass of the whole path over one batch: page table, int32 lengths and split
+plan in one launch (build_decode_metadata: the work of build_block_table and
+get_mla_metadata) and attention with its split merge (mla_decode_paged),
 on inputs resident in HBM.  Default workload: the DeepSeek-V3-shaped decode (bs 64,
 128 heads, q_len 1, L ~ U[1024, 4096], bf16 latent KV 576 wide, 64-token pages in a
 shuffled pool 1.25x the need).  L2 is flushed (512 MB written, then 512 MB read) between timed steps,
@@ -14,7 +15,7 @@ Reported (one JSON line on rank 0):
   roofline     the attention call (decode kernel + merge) against the measured HBM peak:
                algorithmic (KV + Q) bytes / its CUDA-event time;
   e2e          the same metric through the public API with the step's inputs (q,
-               seq_lens, cache_seqlens, req_pool_indices) copied from pinned host memory and
+               seq_lens, req_pool_indices) copied from pinned host memory and
                the outputs (o, lse) copied back inside the timed region, the copies of
                neighbouring steps overlapping the step's compute on their own streams;
   per_config   every workload (tiny, DeepSeek-V3 decode, skewed long context, fp8 cache,
@@ -44,7 +45,7 @@ if ROOT not in sys.path:
 
 METRIC = "paged MLA decode: KV GB/s, TFLOP/s and % roofline; µs per call"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 4  # page table, planner, attention, split merge
+KERNELS_PER_STEP = 3  # metadata (page table, lengths and plan in one launch), attention, split merge
 
 
 def parse_args(argv=None):
@@ -185,8 +186,8 @@ def workload_config(cfg_index, wl, world, flush_mb):
             "head_dim": 576, "head_dim_v": 512,
             "l2": f"flushed between timed steps ({flush_mb} MB written, then another {flush_mb} MB read, "
                   "outside the step events: no input of the step and no dirty line left in L2)",
-            "launch": "each step replays CUDA graphs of the metadata (page table and plan on two "
-                      "streams) and attention calls",
+            "launch": "each step replays CUDA graphs of the metadata call (page table, lengths "
+                      "and plan in one launch) and the attention call",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -259,7 +260,8 @@ def _oracle_rows(wl, rows):
                            wl.cache_seqlens, rows, wl.softmax_scale, wl.causal,
                            kv_is_fp8=wl.is_fp8,
                            descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
-                           descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+                           descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0,
+                           q_is_fp8=wl.q_is_fp8)
     return time.perf_counter() - t0
 
 
@@ -330,12 +332,12 @@ class Case:
     """One workload resident on the device, with its metadata / attention steps captured as
     CUDA graphs the way a serving engine replays them."""
 
-    def __init__(self, cfg, seed, dev, flush_mb):
+    def __init__(self, cfg, seed, dev, flush_mb, q_fp8=False):
         import torch
         import paged_kv_mla_create_b200 as mla
         from paged_kv_mla_create_b200 import workloads as W
         self.mla, self.dev, self.cfg = mla, dev, cfg
-        self.host = host = W.make_workload(cfg, seed=seed)
+        self.host = host = W.make_workload(cfg, seed=seed, q_fp8=q_fp8)
         self.wl = host.to(dev)
         self.kv_bytes, self.q_bytes, self.flops = algorithmic(host)
         bs, q_len, h = host.bs, host.q_len, host.h
@@ -343,34 +345,29 @@ class Case:
         self.bt = torch.empty((bs, host.max_pages), dtype=torch.int32, device=dev)
         self.md = torch.empty((self.parts, 8), dtype=torch.int32, device=dev)
         self.ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
+        self.cl = torch.empty((bs,), dtype=torch.int32, device=dev)
         self.o = torch.empty((bs, q_len, h, 512), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((bs, q_len, h), dtype=torch.float32, device=dev)
-        self.ws = torch.empty((mla.workspace_bytes(bs, q_len, h, self.parts),), dtype=torch.uint8,
+        self.ws = torch.zeros((mla.workspace_bytes(bs, q_len, h, self.parts),), dtype=torch.uint8,
                               device=dev)
         self.flush = torch.empty((flush_mb << 20,), dtype=torch.uint8, device=dev)
         self.flush_rd = torch.ones((flush_mb << 20,), dtype=torch.uint8, device=dev)
-        self.side = torch.cuda.Stream(dev)
 
     def flush_l2(self, i):
         self.flush.fill_(i & 0xFF)
         self.flush_rd.max()   # evicts the written lines while still outside the timed region
 
     def metadata(self, w):
-        import torch
+        """Page table, int32 cache_seqlens and split plan: one launch."""
         host = self.host
-        # the page table and the plan are independent: the plan runs on a side stream
-        cur = torch.cuda.current_stream(self.dev)
-        self.side.wait_stream(cur)
-        with torch.cuda.stream(self.side):
-            self.mla.get_mla_metadata(w.cache_seqlens, host.q_len * host.h, 1, host.is_fp8,
-                                      out=(self.md, self.ns))
-        self.mla.build_block_table(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
-                                   seq_len_add=host.num_draft_tokens, out=self.bt)
-        cur.wait_stream(self.side)
+        self.mla.build_decode_metadata(w.req_to_token, w.req_pool_indices, w.seq_lens, host.max_pages,
+                                       host.q_len * host.h, 1, host.is_fp8,
+                                       seq_len_add=host.num_draft_tokens,
+                                       out=(self.bt, self.cl, self.md, self.ns))
 
     def attention(self, w, o=None, lse=None):
         host = self.host
-        self.mla.mla_decode_paged(w.q, w.kv_cache, self.bt, w.cache_seqlens, 512, self.md, self.ns,
+        self.mla.mla_decode_paged(w.q, w.kv_cache, self.bt, self.cl, 512, self.md, self.ns,
                                   host.softmax_scale, host.causal, w.descale_q, w.descale_k,
                                   out=self.o if o is None else o, lse=self.lse if lse is None else lse,
                                   workspace=self.ws)
@@ -440,16 +437,16 @@ class Case:
 
     def time_e2e(self, steps):
         """The same step end to end through the public API, from pinned host buffers: step k's
-        inputs (q, seq_lens, cache_seqlens, req_pool_indices) are copied in on a copy stream
+        inputs (q, seq_lens, req_pool_indices) are copied in on a copy stream
         while step k - 1 computes, and step k's o and lse are copied out on another while step
         k + 1 computes (two device buffer sets).  Every step's copies lie inside the timed
         region, which runs from the first copy in to the last copy out.  No L2 flush: the KV
-        cache every step streams is larger than L2.  Returns (ms per step, h2d, d2h bytes)."""
+        cache every step streams is larger than L2.  (cache_seqlens is not an input: the
+        metadata launch derives it from seq_lens.)  Returns (ms per step, h2d, d2h bytes)."""
         import dataclasses
         import torch
         host, wl, dev = self.host, self.wl, self.dev
-        pin = [t.pin_memory() for t in (host.q, host.seq_lens, host.cache_seqlens,
-                                        host.req_pool_indices)]
+        pin = [t.pin_memory() for t in (host.q, host.seq_lens, host.req_pool_indices)]
         outs_h = [(torch.empty(self.o.shape, dtype=self.o.dtype, pin_memory=True),
                    torch.empty(self.lse.shape, dtype=self.lse.dtype, pin_memory=True)) for _ in range(2)]
         ins_d, outs_d, wls = [], [], []
@@ -457,8 +454,7 @@ class Case:
             d = [torch.empty_like(t, device=dev) for t in pin]
             ins_d.append(d)
             outs_d.append((torch.empty_like(self.o), torch.empty_like(self.lse)))
-            wls.append(dataclasses.replace(wl, q=d[0], seq_lens=d[1], cache_seqlens=d[2],
-                                           req_pool_indices=d[3]))
+            wls.append(dataclasses.replace(wl, q=d[0], seq_lens=d[1], req_pool_indices=d[2]))
         h2d = sum(t.numel() * t.element_size() for t in pin)
         d2h = sum(t.numel() * t.element_size() for t in outs_h[0])
         comp = torch.cuda.current_stream(dev)
@@ -505,9 +501,8 @@ class Case:
 
 
 def config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src):
-    from paged_kv_mla_create_b200.workloads import CONFIGS
     attn_s = attn_ms * 1e-3
-    return {"workload": CONFIGS[case.cfg]["name"], "us_per_call": attn_ms * 1e3,
+    return {"workload": case.host.name, "us_per_call": attn_ms * 1e3,
             "metadata_us": meta_ms * 1e3, "us_per_step": step_ms * 1e3,
             "kv_gbs_per_call": case.kv_bytes / attn_s / 1e9, "tflops": case.flops / attn_s / 1e12,
             "kv_bytes": case.kv_bytes, "q_bytes": case.q_bytes, "flops": case.flops,
@@ -552,17 +547,18 @@ def run_b200(args):
     # every other workload, with a short timed run each (its own clock record)
     per_config = {str(args.config): head}
     if not args.no_per_config:
-        for cfg in (1, 2, 3, 4, 5):
-            if cfg == args.config:
+        # the five workloads, and the fp8-cache one with e4m3 queries (the backend's fp8 recipe)
+        for cfg, q8 in ((1, False), (2, False), (3, False), (4, False), (4, True), (5, False)):
+            if cfg == args.config and not q8:
                 continue
-            c = Case(cfg, replica_seed(cfg, rank), dev, args.flush_mb)
+            c = Case(cfg, replica_seed(cfg, rank), dev, args.flush_mb, q_fp8=q8)
             sm, am, mm, ck = c.time_steps(max(1, min(K, args.per_config_steps)), max(3, min(args.warmup, 5)),
                                           world, ClockSampler(gpu_id_for(dev)))
             e = mla.read_device_error(dev)
             sm, am, mm, e = reduce_max_over_ranks([sm, am, mm, float(e)], dev, world)
             if e:
                 raise RuntimeError(f"device error word {int(e)} after workload {cfg}")
-            per_config[str(cfg)] = config_entry(c, sm, am, mm, ck, peaks, peak_src)
+            per_config[f"{cfg}q8" if q8 else str(cfg)] = config_entry(c, sm, am, mm, ck, peaks, peak_src)
             del c
             torch.cuda.empty_cache()
 

@@ -60,7 +60,8 @@ enum {
     MLA_DTYPE_BF16 = 0,
     MLA_DTYPE_FP8_E4M3 = 1,    /* OCP e4m3 "fn": no infinities, S.1111.111 = NaN */
     MLA_DTYPE_INT32 = 2,
-    MLA_DTYPE_INT64 = 3
+    MLA_DTYPE_INT64 = 3,
+    MLA_DTYPE_FP8_E5M2 = 4     /* OCP e5m2: exponent 31 holds infinities and NaNs   */
 };
 
 /* Bits of the sticky device error word (mla_read_device_error). */
@@ -70,9 +71,12 @@ enum {
     MLA_DEVERR_LEN_OUT_OF_RANGE = 4,   /* a length exceeds the table / req_to_token width: clamped     */
     MLA_DEVERR_BAD_METADATA = 8,       /* a scheduler row is not a valid cursor range: part skipped    */
     MLA_DEVERR_WAIT_TIMEOUT = 16,      /* a pipeline wait exceeded its bound: the CTA gave up          */
-    MLA_DEVERR_Q_RANGE = 32,           /* e4m3 cache: a q value beyond the f16 range (|q| > 65504)     */
-    MLA_DEVERR_SLOT_INVALID = 64       /* page table: a req_to_token slot read for page p is negative    */
+    MLA_DEVERR_Q_RANGE = 32,           /* 8-bit cache, bf16 q: a q value beyond f16's range (> 65504)  */
+    MLA_DEVERR_SLOT_INVALID = 64,      /* page table: a req_to_token slot read for page p is negative    */
                                        /* (entry -1) or not the first slot of a page (slot % 64 != 0)  */
+    MLA_DEVERR_WORKSPACE_STATE = 128,  /* decode: a workspace arrival word was not zero at the call's  */
+                                       /* start (workspace not zero-filled before its first use)       */
+    MLA_DEVERR_SLOT_OUT_OF_RANGE = 256 /* KV write: cache_loc[i] not a pool row: that token skipped    */
 };
 
 typedef struct CUstream_st* mla_stream_t;  /* identical to cudaStream_t */
@@ -162,8 +166,32 @@ MLA_API mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t 
                                   mla_stream_t stream);
 
 /*
- * Bytes of workspace mla_decode_paged needs: partial outputs fp32
- * [(bs + num_sm_parts) * q_len * h_q, 512] and their log-sum-exps, 256-byte aligned.
+ * The whole per-batch metadata step in one launch: mla_build_block_table,
+ * the int32 cache_seqlens the attention call takes (flashmla_backend.py,
+ * init_forward_metadata: seq_lens.to(torch.int32), plus num_draft_tokens in the
+ * target-verify branch) and mla_get_mla_metadata over those lengths.
+ *
+ * Arguments are those of mla_build_block_table followed by those of
+ * mla_get_mla_metadata; the lengths the plan uses are seq_lens[b] + seq_len_add.
+ *   cache_seqlens          int32 [bs], written with seq_lens[b] + seq_len_add; may be NULL
+ * block_table, tile_scheduler_metadata and num_splits are bit-identical to what the two
+ * separate calls write (one CTA plans while the others fill the table).  Errors and
+ * device checks are those of the two calls.
+ */
+MLA_API mla_status_t mla_build_decode_metadata(
+    const int32_t* req_to_token, int64_t req_to_token_rows, int64_t req_to_token_stride,
+    const void* req_pool_indices, int32_t rpi_dtype, const void* seq_lens, int32_t seq_lens_dtype,
+    int32_t seq_len_add, int32_t bs, int32_t* block_table, int64_t block_table_stride,
+    int32_t max_pages, int32_t page_size, int32_t fill_tail, int32_t num_heads_per_head_k,
+    int32_t num_heads_k, int32_t is_fp8_kvcache, int32_t sm_count, int32_t* cache_seqlens,
+    int32_t* tile_scheduler_metadata, int32_t* num_splits, mla_stream_t stream);
+
+/*
+ * Bytes of workspace mla_decode_paged needs, 256-byte aligned parts in this order:
+ *   arrival words  int32 [bs, cdiv(q_len * h_q, 128), 2]: split pieces of a request count
+ *                  their arrival here, and the last to arrive merges the request's rows
+ *                  (requests of up to 4 pieces); every completed call leaves them zero;
+ *   partial outputs fp32 [(bs + num_sm_parts) * q_len * h_q, 512] and their log-sum-exps.
  * Pure host function; returns 0 on a non-positive argument.
  */
 MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q, int32_t num_sm_parts);
@@ -181,18 +209,22 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *   v_j = k_j[0:512];  s_j = softmax_scale * descale_q * <q[b,i,h,:], k_j>;
  *   lse = ln sum_j exp(s_j);  o = sum_j exp(s_j - lse) v_j.
  *   A row with no allowed key gets o = 0 and lse = -inf.
- *   Arithmetic: S in fp32 from bf16 products (bf16 cache) or f16 products (e4m3 cache:
- *   every e4m3 value is exact in f16; a bf16 q value is exact in f16 when its magnitude
+ *   Arithmetic: S in fp32 from bf16 products (bf16 cache) or f16 products (8-bit cache with
+ *   bf16 q: every e4m3 and e5m2 value is exact in f16; a bf16 q value is exact in f16 when its magnitude
  *   lies in [2^-14, 65504] or it is zero, while magnitudes in [2^-24, 2^-14) keep only
  *   the bits of an f16 subnormal and smaller ones round to zero, an error far below the
  *   attention tolerance; |q| > 65504 records MLA_DEVERR_Q_RANGE and o is undefined); P
- *   rounded to bf16 (f16 with an e4m3 cache) for the P V product; O accumulated in fp32.
+ *   rounded to bf16 (f16 with an 8-bit cache) for the P V product; O accumulated in fp32.
+ *   With e4m3 q, S is fp32 from exact e4m3 x e4m3 products.
  *
  *   q                 bf16 [bs, q_len, h_q, head_dim], contiguous; q_len * h_q must not
  *                     exceed 65535 * 128 (MLA_ERR_UNSUPPORTED)
- *   q_dtype           MLA_DTYPE_BF16
+ *   q_dtype           MLA_DTYPE_BF16, or MLA_DTYPE_FP8_E4M3 with an e4m3 cache (the backend
+ *                     page's fp8 branch: q quantised with scaled_fp8_quant(q, k_scale),
+ *                     descale_q = descale_k = k_scale); S then runs on e4m3 x e4m3 tensor
+ *                     cores, PV on f16.  e4m3 q with another cache: MLA_ERR_UNSUPPORTED
  *   head_dim          576 (kv_lora_rank 512 + qk_rope_head_dim 64); head_dim_v 512
- *   k_cache           [num_pages, page_size, head_dim] bf16 or e4m3 (kv_dtype), contiguous;
+ *   k_cache           [num_pages, page_size, head_dim] bf16, e4m3 or e5m2 (kv_dtype), contiguous;
  *                     every value must be finite (tail rows of a page are read and masked)
  *   page_size         64
  *   block_table       int32 [bs, block_table_stride]; entries p < cdiv(L, 64) are read
@@ -203,16 +235,20 @@ MLA_API size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q
  *                     mla_num_sm_parts(sm_count, q_len * h_q, 1)
  *   softmax_scale     host float (1/sqrt(192) for DeepSeek-V3)
  *   causal            0 or 1
- *   descale_q, descale_k  device fp32 [1]; NULL means 1.0.  descale_k scales the fp8
+ *   descale_q, descale_k  device fp32 [1]; NULL means 1.0.  descale_k scales the 8-bit
  *                     cache values and must be NULL with a bf16 cache (the backend passes
  *                     the descales only with an fp8 cache), else MLA_ERR_INVALID_ARG;
  *                     descale_q scales q.
  *   out               bf16 [bs, q_len, h_q, 512] (written)
  *   lse               fp32 [bs, q_len, h_q] natural-log log-sum-exp (written)
  *   workspace         at least mla_decode_workspace_bytes(bs, q_len, h_q, num_sm_parts)
- *                     bytes, 256-byte aligned; its contents need no initialisation and are
- *                     undefined after the call (the merge may drop the split partials'
- *                     L2 lines without writing them back)
+ *                     bytes, 256-byte aligned, zero-filled before its first use: its leading
+ *                     arrival words must be zero when a call starts, and every completed call
+ *                     leaves them zero again, so a workspace is zero-filled once and then
+ *                     reused (after a call that recorded MLA_DEVERR_WAIT_TIMEOUT or
+ *                     MLA_DEVERR_WORKSPACE_STATE, zero-fill it again).  The partial-output
+ *                     part needs no initialisation and is undefined after the call (the merge
+ *                     may drop its L2 lines without writing them back)
  * Calls on the same workspace that overlap on the GPU race; use one workspace per stream.
  * The first call on a device also sets the kernel's shared-memory limit (a host-side
  * attribute; no allocation).
@@ -227,6 +263,32 @@ MLA_API mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs
                               int32_t causal, const float* descale_q, const float* descale_k,
                               void* out, float* lse, void* workspace, size_t workspace_bytes,
                               mla_stream_t stream);
+
+/*
+ * KV-cache write (flashmla_backend.py, forward_decode / forward_extend:
+ * token_to_kv_pool.set_kv_buffer(layer, cache_loc, k, v) before attention).  For every new
+ * token i, pool row cache_loc[i] receives k[i, 0:576], the latent row (kv_lora_rank 512 +
+ * qk_rope_head_dim 64); in MLA the value is the first 512 columns of that row, so v is not
+ * passed.  A bf16 pool stores the row bit for bit; an fp8 pool (MLA_DTYPE_FP8_E4M3 or
+ * MLA_DTYPE_FP8_E5M2, the two fp8 types the backend's __init__ accepts) stores
+ * x = k / k_scale, one correctly rounded single-precision division (x = k when k_scale is
+ * NULL), rounded to the nearest code, ties to even, magnitudes beyond the largest finite
+ * value saturating to it.
+ *
+ *   kv_cache      the pool [num_slots, 576] of kv_dtype, contiguous; 16-byte aligned (bf16)
+ *                 or 8-byte aligned (fp8)
+ *   cache_loc     [n_tokens] int32 or int64 (loc_dtype): each token's pool row
+ *   k             bf16 [n_tokens, k_row_stride] (elements), 16-byte aligned;
+ *                 k_row_stride >= 576 and a multiple of 8
+ *   k_scale       device fp32 [1] or NULL; must be NULL for a bf16 pool
+ * Rows not listed are untouched.  A cache_loc outside [0, num_slots) skips that token and
+ * sets MLA_DEVERR_SLOT_OUT_OF_RANGE.  Two tokens with the same slot race (one wins).
+ * n_tokens == 0 returns MLA_OK and launches nothing.
+ */
+MLA_API mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slots,
+                                       const void* cache_loc, int32_t loc_dtype, int32_t n_tokens,
+                                       const void* k, int64_t k_row_stride, const float* k_scale,
+                                       mla_stream_t stream);
 
 /*
  * Read and clear the sticky device error word of the current device (a bitwise OR of
@@ -253,8 +315,10 @@ MLA_API mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t strea
  * rejected with MLA_ERR_WORKSPACE before anything is launched; the five DeepSeek-V3-shaped
  * workloads of this project (up to bs 128 x 128 heads, or bs 32 x 4 x 128 rows) fit.
  *
- * All calls share the one array and it keeps whatever the last call left in it; the
- * kernels write every scratch value before reading it, so nothing needs clearing.  Calls
+ * All calls share the one array and it keeps whatever the last call left in it: each call
+ * first clears the array's leading arrival words (the only scratch that must start at zero;
+ * an asynchronous memset on `stream`, no allocation), and its kernels write every other
+ * scratch value before reading it.  Calls
  * whose execution overlaps on the GPU (on different streams, or from different threads)
  * race on the array and corrupt each other's results: serialise them.
  *

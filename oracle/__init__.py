@@ -66,6 +66,12 @@ def _load():
     lib.oracle_merge_states.restype = None
     lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
     lib.oracle_e4m3_to_double.restype = D
+    lib.oracle_e5m2_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e5m2_to_double.restype = D
+    lib.oracle_quantize_fp8.argtypes = [D, I32]
+    lib.oracle_quantize_fp8.restype = ctypes.c_uint8
+    lib.oracle_set_kv_buffer.argtypes = [P, I32, I64, I64, P, I64, P, I64, I32, ctypes.c_float]
+    lib.oracle_set_kv_buffer.restype = None
     lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_double.restype = D
     lib.oracle_num_threads.argtypes = []
@@ -78,7 +84,7 @@ def _np(x, dtype):
     """Contiguous numpy array of the given dtype from a numpy array or CPU torch tensor."""
     if hasattr(x, "detach"):
         x = x.detach().cpu()
-        if str(x.dtype) in ("torch.bfloat16", "torch.float8_e4m3fn"):
+        if str(x.dtype) in ("torch.bfloat16", "torch.float8_e4m3fn", "torch.float8_e5m2"):
             import torch
             x = x.view(torch.uint16 if x.dtype == torch.bfloat16 else torch.uint8)
         x = x.numpy()
@@ -100,6 +106,43 @@ def e4m3_to_double(code: int) -> float:
 
 def bf16_to_double(bits: int) -> float:
     return _load().oracle_bf16_to_double(bits)
+
+
+def e5m2_to_double(code: int) -> float:
+    return _load().oracle_e5m2_to_double(code)
+
+
+FP8_FORMATS = {"e4m3": 1, "e5m2": 2}
+
+
+def quantize_fp8(x: float, fmt: str = "e4m3") -> int:
+    """The code of x rounded to the 8-bit format (nearest, ties to even, saturating)."""
+    return int(_load().oracle_quantize_fp8(float(x), FP8_FORMATS[fmt]))
+
+
+def _kv_format(kv_cache, kv_is_fp8):
+    dt = str(getattr(kv_cache, "dtype", ""))
+    if dt == "torch.float8_e5m2":
+        return 2
+    return 1 if kv_is_fp8 else 0
+
+
+def set_kv_buffer(pool, cache_loc, k, k_scale=None):
+    """Write the new tokens' rows k [n, dim] (bf16) at pool rows cache_loc [n]; pool is a
+    torch tensor [slots, dim] of bf16, float8_e4m3fn or float8_e5m2 (modified in place,
+    CPU).  An fp8 pool stores k / k_scale rounded to its format."""
+    import torch
+    fmt = {torch.bfloat16: 0, torch.float8_e4m3fn: 1, torch.float8_e5m2: 2}[pool.dtype]
+    raw = pool.view(torch.uint16 if fmt == 0 else torch.uint8)
+    assert raw.is_contiguous()
+    arr = raw.numpy()   # shares memory with pool
+    loc = _np(cache_loc, np.int64).reshape(-1)
+    kb = _np(k, np.uint16)
+    dim = arr.shape[-1]
+    _load().oracle_set_kv_buffer(_ptr(arr), fmt, arr.size // dim, dim, _ptr(loc), loc.shape[0], _ptr(kb),
+                                 kb.shape[-1], int(k_scale is not None),
+                                 float(k_scale) if k_scale is not None else 1.0)
+    return pool
 
 
 def build_block_table(req_to_token, req_pool_indices, seq_lens, max_pages: int,
@@ -136,14 +179,15 @@ def mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, 
                     key_begin=None, key_end=None, q_is_fp8: bool = False):
     """Attention for the flat rows (b * q_len + i) * h + head of q [bs, q_len, h, dq].
 
-    kv_cache is the token-slot pool (any shape whose last dim is dq; bf16 or e4m3
-    torch tensors, or their raw uint16 / uint8 bits); q is bf16, or e4m3 codes with
+    kv_cache is the token-slot pool (any shape whose last dim is dq; bf16, e4m3 or e5m2
+    torch tensors, or the raw uint16 / uint8 bits of bf16 / e4m3 ones); q is bf16, or e4m3 codes with
     q_is_fp8 (descale_q then being the scale q was quantised with).  Returns
     (o [n, dv] fp64, lse [n] fp64).
     """
     qb = _np(q, np.uint8 if q_is_fp8 else np.uint16)
     bs, q_len, h, dq = qb.shape
-    kv = _np(kv_cache, np.uint8 if kv_is_fp8 else np.uint16).reshape(-1, dq)
+    kv_format = _kv_format(kv_cache, kv_is_fp8)
+    kv = _np(kv_cache, np.uint8 if kv_format else np.uint16).reshape(-1, dq)
     r2t = _np(req_to_token, np.int32)
     rpi = _np(req_pool_indices, np.int64)
     sl = _np(cache_seqlens, np.int32)
@@ -154,7 +198,7 @@ def mla_decode_rows(q, kv_cache, req_to_token, req_pool_indices, cache_seqlens, 
     o = np.empty((n, head_dim_v), dtype=np.float64)
     lse = np.empty((n,), dtype=np.float64)
     rc = _load().oracle_mla_decode_rows(
-        _ptr(qb), int(q_is_fp8), _ptr(kv), int(kv_is_fp8), float(descale_q), float(descale_k), _ptr(r2t),
+        _ptr(qb), int(q_is_fp8), _ptr(kv), kv_format, float(descale_q), float(descale_k), _ptr(r2t),
         r2t.shape[1], _ptr(rpi), _ptr(sl), _ptr(kb) if kb is not None else None,
         _ptr(ke) if ke is not None else None, bs, q_len, h, dq, head_dim_v, float(softmax_scale),
         int(causal), n, _ptr(rows), _ptr(o), _ptr(lse))

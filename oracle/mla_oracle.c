@@ -27,6 +27,11 @@
  *   oracle_merge_states       the log-sum-exp merge of partial attention states
  *                             (flashinfer_backend.py, forward_extend: merge_state of a
  *                             ragged and a paged partial result).
+ *   oracle_set_kv_buffer      flashmla_backend.py, forward_decode / forward_extend
+ *                             (token_to_kv_pool.set_kv_buffer(layer, cache_loc, k, v): the
+ *                             new tokens' 576-wide latent rows written at their pool slots
+ *                             before attention; an fp8 pool, float8_e4m3fn or float8_e5m2 as
+ *                             __init__ lists them, stores k / k_scale rounded to its format).
  */
 #include <math.h>
 #include <omp.h>
@@ -57,10 +62,59 @@ static double e4m3_bits_to_double(uint8_t bits) {
     return sign ? -v : v;
 }
 
+/* OCP float8 e5m2: 1 sign, 5 exponent (bias 15), 2 mantissa bits, subnormals when the
+ * exponent field is 0; exponent field 31 holds infinities (mantissa 0) and NaNs. */
+static double e5m2_bits_to_double(uint8_t bits) {
+    int sign = bits >> 7;
+    int e = (bits >> 2) & 0x1F;
+    int m = bits & 0x3;
+    double v;
+    if (e == 0x1F) v = m == 0 ? INFINITY : NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -16);           /* m/4 * 2^(1-15) */
+    else
+        v = ldexp((double)(4 + m), e - 17);  /* (1 + m/4) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* Element of an 8-bit cache: format 1 = e4m3, 2 = e5m2. */
+static double fp8_bits_to_double(uint8_t bits, int format) {
+    return format == 2 ? e5m2_bits_to_double(bits) : e4m3_bits_to_double(bits);
+}
+
+/*
+ * Round x to the 8-bit format (1 = e4m3, 2 = e5m2) by brute force: among the codes of x's
+ * sign, the one whose value is nearest to x, ties to the code with an even mantissa (even
+ * code); magnitudes beyond the largest finite value give that value (saturation); NaN gives
+ * the format's NaN code.
+ */
+static uint8_t quantize_fp8(double x, int format) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    int best = -1, top = 0;
+    double best_err = INFINITY;
+    for (int code = 0; code < 0x80; ++code)   /* the largest finite code of the format */
+        if (isfinite(fp8_bits_to_double((uint8_t)code, format))) top = code;
+    if (a >= fp8_bits_to_double((uint8_t)top, format)) return (uint8_t)(sign | top);
+    for (int code = 0; code < 0x80; ++code) {
+        double v = fp8_bits_to_double((uint8_t)code, format);
+        if (!isfinite(v)) continue;
+        double err = fabs(v - a);
+        if (err < best_err || (err == best_err && (code & 1) == 0)) {
+            best = code;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
 /* Threads the OpenMP loops use (the host's cores unless OMP_NUM_THREADS says otherwise). */
 int oracle_num_threads(void) { return omp_get_max_threads(); }
 
 double oracle_e4m3_to_double(uint8_t bits) { return e4m3_bits_to_double(bits); }
+double oracle_e5m2_to_double(uint8_t bits) { return e5m2_bits_to_double(bits); }
+uint8_t oracle_quantize_fp8(double x, int format) { return quantize_fp8(x, format); }
 double oracle_bf16_to_double(uint16_t bits) { return bf16_bits_to_double(bits); }
 
 static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -161,14 +215,14 @@ void oracle_get_mla_metadata(const int32_t* cache_seqlens, int64_t bs, int64_t n
  * restricted to the causally allowed keys.  The allowed keys are j < lim with
  * lim = L - q_len + i + 1 under causal (the draft tokens' own KV is the last q_len
  * positions of the cache, written before attention), lim = L otherwise.
- *   k_j = KV[req_to_token[rpi[b], j], 0:dq] * descale_k   (fp64, exact)
+ *   k_j = KV[req_to_token[rpi[b], j], 0:dq] (* descale_k for an fp8 cache)   (fp64, exact)
  *   v_j = k_j[0:dv]
  *   s_j = softmax_scale * descale_q * sum_d q[d] * k_j[d]
  *   lse = m + ln(sum_j exp(s_j - m)),  m = max_j s_j
  *   o   = sum_j exp(s_j - lse) * v_j
  * With no allowed key: o = 0 and lse = -inf.
  */
-static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int kv_is_fp8,
+static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int kv_format,
                        double descale_q, double descale_k, const int32_t* r2t_row, int64_t j_begin,
                        int64_t j_end, int64_t dq, int64_t dv, double softmax_scale, double* o,
                        double* lse, double* s_buf) {
@@ -187,7 +241,7 @@ static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int k
         int64_t slot = r2t_row[j_begin + t];
         double acc = 0.0;
         for (int64_t d = 0; d < dq; ++d) {
-            double kd = kv_is_fp8 ? e4m3_bits_to_double(kv[slot * dq + d]) * descale_k
+            double kd = kv_format ? fp8_bits_to_double(kv[slot * dq + d], kv_format) * descale_k
                                   : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);
             acc += qd[d] * kd;
         }
@@ -202,7 +256,7 @@ static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int k
         int64_t slot = r2t_row[j_begin + t];
         double w = exp(s_buf[t] - l);
         for (int64_t d = 0; d < dv; ++d) {
-            double vd = kv_is_fp8 ? e4m3_bits_to_double(kv[slot * dq + d]) * descale_k
+            double vd = kv_format ? fp8_bits_to_double(kv[slot * dq + d], kv_format) * descale_k
                                   : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);
             o[d] += w * vd;
         }
@@ -215,13 +269,13 @@ static void attend_row(const void* q_row, int q_is_fp8, const uint8_t* kv, int k
  * into the [bs, q_len, h] grid; o_out is [n_rows, dv] and lse_out [n_rows].
  * key_begin / key_end (nullable, indexed by b) restrict request b's keys to a range
  * before the causal limit is applied; null means the whole [0, L).
- * kv is the flat token-slot pool [num_slots, dq] of bf16 bits (kv_is_fp8 = 0) or
- * e4m3 bytes (kv_is_fp8 = 1); q is [bs, q_len, h, dq] of bf16 bits (q_is_fp8 = 0) or e4m3
+ * kv is the flat token-slot pool [num_slots, dq] of bf16 bits (kv_format = 0), e4m3
+ * bytes (kv_format = 1) or e5m2 bytes (kv_format = 2); q is [bs, q_len, h, dq] of bf16 bits (q_is_fp8 = 0) or e4m3
  * bytes (q_is_fp8 = 1: the flash_mla_with_kvcache call of the FlashMLA backend page, with q
  * quantised by scaled_fp8_quant and descale_q its scale).  Returns 0, or -1 when the query
  * width exceeds 1024.
  */
-int oracle_mla_decode_rows(const void* q, int q_is_fp8, const void* kv, int kv_is_fp8, double descale_q,
+int oracle_mla_decode_rows(const void* q, int q_is_fp8, const void* kv, int kv_format, double descale_q,
                            double descale_k, const int32_t* req_to_token, int64_t r2t_stride,
                            const int64_t* req_pool_indices, const int32_t* cache_seqlens,
                            const int64_t* key_begin, const int64_t* key_end, int64_t bs,
@@ -252,7 +306,7 @@ int oracle_mla_decode_rows(const void* q, int q_is_fp8, const void* kv, int kv_i
             if (j1 > lim) j1 = lim;
             const void* q_row = q_is_fp8 ? (const void*)((const uint8_t*)q + flat * dq)
                                          : (const void*)((const uint16_t*)q + flat * dq);
-            attend_row(q_row, q_is_fp8, (const uint8_t*)kv, kv_is_fp8, descale_q, descale_k,
+            attend_row(q_row, q_is_fp8, (const uint8_t*)kv, kv_format, descale_q, descale_k,
                        req_to_token + req_pool_indices[b] * r2t_stride, j0, j1, dq, dv,
                        softmax_scale, o_out + r * dv, lse_out + r, s_buf);
         }
@@ -284,4 +338,30 @@ void oracle_merge_states(int64_t n, int64_t dv, const double* o_parts, const dou
         for (int64_t d = 0; d < dv; ++d) o[d] += w * o_parts[k * dv + d];
     }
     *lse = l;
+}
+
+/*
+ * KV-cache write: for every new token i, row cache_loc[i] of the pool [num_slots, dim]
+ * receives k[i, 0:dim] (k is bf16 bits with row stride k_stride).  A bf16 pool (format 0)
+ * stores the bits as they are.  An fp8 pool (format 1 = e4m3, 2 = e5m2) stores
+ * quantize_fp8(x), with x = k / k_scale evaluated in float32 (one correctly rounded
+ * division) when has_scale, else k itself.  Slots outside [0, num_slots) are skipped.
+ */
+void oracle_set_kv_buffer(void* pool, int format, int64_t num_slots, int64_t dim,
+                          const int64_t* cache_loc, int64_t n_tokens, const uint16_t* k,
+                          int64_t k_stride, int has_scale, float k_scale) {
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int64_t slot = cache_loc[i];
+        if (slot < 0 || slot >= num_slots) continue;
+        for (int64_t d = 0; d < dim; ++d) {
+            uint16_t bits = k[i * k_stride + d];
+            if (format == 0) {
+                ((uint16_t*)pool)[slot * dim + d] = bits;
+            } else {
+                float x = (float)bf16_bits_to_double(bits);
+                if (has_scale) x = x / k_scale;
+                ((uint8_t*)pool)[slot * dim + d] = quantize_fp8((double)x, format);
+            }
+        }
+    }
 }

@@ -28,14 +28,17 @@ import torch
 from . import build as _build
 
 __all__ = [
-    "build_block_table", "get_mla_metadata", "mla_decode_paged", "flash_mla_with_kvcache",
+    "build_block_table", "get_mla_metadata", "build_decode_metadata", "mla_decode_paged",
+    "flash_mla_with_kvcache", "set_kv_buffer",
     "num_sm_parts", "workspace_bytes", "read_device_error", "library", "MlaError",
 ]
 
 PAGE_SIZE = 64
 _STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_CUDA",
            4: "MLA_ERR_DEVICE_CHECK", 5: "MLA_ERR_WORKSPACE"}
-DTYPE_BF16, DTYPE_FP8_E4M3, DTYPE_INT32, DTYPE_INT64 = 0, 1, 2, 3
+DTYPE_BF16, DTYPE_FP8_E4M3, DTYPE_INT32, DTYPE_INT64, DTYPE_FP8_E5M2 = 0, 1, 2, 3, 4
+_CACHE_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float8_e4m3fn: DTYPE_FP8_E4M3,
+                 torch.float8_e5m2: DTYPE_FP8_E5M2}
 
 _lib = None
 
@@ -70,11 +73,16 @@ def library() -> ctypes.CDLL:
     lib.mla_num_sm_parts.restype = I32
     lib.mla_get_mla_metadata.argtypes = [P, I32, I32, I32, I32, I32, P, P, P]
     lib.mla_get_mla_metadata.restype = I32
+    lib.mla_build_decode_metadata.argtypes = [P, I64, I64, P, I32, P, I32, I32, I32, P, I64, I32,
+                                              I32, I32, I32, I32, I32, I32, P, P, P, P]
+    lib.mla_build_decode_metadata.restype = I32
     lib.mla_decode_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.mla_decode_workspace_bytes.restype = SZ
     lib.mla_decode_paged.argtypes = [P, I32, I32, I32, I32, I32, I32, P, I32, I64, I32, P, I64,
                                      I32, P, P, I32, P, F, I32, P, P, P, P, P, SZ, P]
     lib.mla_decode_paged.restype = I32
+    lib.mla_set_kv_buffer.argtypes = [P, I32, I64, P, I32, I32, P, I64, P, P]
+    lib.mla_set_kv_buffer.restype = I32
     lib.mla_read_device_error.argtypes = [ctypes.POINTER(I32), P]
     lib.mla_read_device_error.restype = I32
     _lib = lib
@@ -123,6 +131,8 @@ def num_sm_parts(num_heads_per_head_k: int, num_heads_k: int = 1,
 
 
 def workspace_bytes(bs: int, q_len: int, h_q: int, parts: int) -> int:
+    """Bytes of the attention workspace; allocate it zero-filled (torch.zeros) once, then
+    reuse it: every completed call leaves its leading arrival words zero."""
     return int(library().mla_decode_workspace_bytes(bs, q_len, h_q, parts))
 
 
@@ -185,6 +195,49 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, num_heads_per_head_k: int,
     return md, ns
 
 
+def build_decode_metadata(req_to_token: torch.Tensor, req_pool_indices: torch.Tensor,
+                          seq_lens: torch.Tensor, max_seqlen_pad: int, num_heads_per_head_k: int,
+                          num_heads_k: int = 1, is_fp8_kvcache: bool = False, seq_len_add: int = 0,
+                          num_parts: Optional[int] = None, fill_tail: bool = True,
+                          out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]] = None):
+    """The per-batch metadata in one launch: (block_table int32 [bs, max_seqlen_pad],
+    cache_seqlens int32 [bs] = seq_lens + seq_len_add, tile_scheduler_metadata int32
+    [num_sm_parts, 8], num_splits int32 [bs + 1]) -- what build_block_table, the int32 cast
+    of the lengths and get_mla_metadata give."""
+    _require_cuda(req_to_token, req_pool_indices, seq_lens)
+    if req_to_token.dtype != torch.int32 or req_to_token.dim() != 2 or req_to_token.stride(1) != 1:
+        raise ValueError("req_to_token must be a row-major int32 matrix")
+    if num_heads_per_head_k <= 0 or num_heads_k <= 0:
+        raise ValueError("num_heads_per_head_k and num_heads_k must be positive")
+    dev = req_to_token.device
+    bs = int(req_pool_indices.shape[0])
+    if num_parts is not None:
+        sms = 2 * (-(-num_heads_per_head_k // 128)) * num_heads_k * int(num_parts)
+    else:
+        sms = sm_count(dev)
+    parts = num_sm_parts(num_heads_per_head_k, num_heads_k, sms)
+    if out is None:
+        bt = torch.empty((bs, max_seqlen_pad), dtype=torch.int32, device=dev)
+        cl = torch.empty((bs,), dtype=torch.int32, device=dev)
+        md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
+        ns = torch.empty((bs + 1,), dtype=torch.int32, device=dev)
+    else:
+        bt, cl, md, ns = out
+    if bt.dtype != torch.int32 or bt.dim() != 2 or bt.stride(1) != 1:
+        raise ValueError("block_table must be a row-major int32 matrix")
+    if md.shape[0] != parts or ns.numel() != bs + 1 or (cl is not None and cl.numel() != bs):
+        raise ValueError("out tensors do not match the metadata's shapes")
+    rpi = req_pool_indices.contiguous()
+    sl = seq_lens.contiguous()
+    _check(library().mla_build_decode_metadata(
+        _ptr(req_to_token), req_to_token.shape[0], req_to_token.stride(0), _ptr(rpi),
+        _index_dtype(rpi), _ptr(sl), _index_dtype(sl), int(seq_len_add), bs, _ptr(bt), bt.stride(0),
+        int(max_seqlen_pad), PAGE_SIZE, int(bool(fill_tail)), int(num_heads_per_head_k),
+        int(num_heads_k), int(bool(is_fp8_kvcache)), sms, _ptr(cl), _ptr(md), _ptr(ns),
+        _stream(dev)), "mla_build_decode_metadata")
+    return bt, cl, md, ns
+
+
 def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
                      cache_seqlens: torch.Tensor, head_dim_v: int,
                      tile_scheduler_metadata: torch.Tensor, num_splits: torch.Tensor,
@@ -193,26 +246,24 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
                      descale_k: Optional[torch.Tensor] = None,
                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None):
-    """Paged MLA attention.  q bf16 [bs, q_len, h_q, 576]; k_cache bf16 or float8_e4m3fn
-    with 576-wide token rows grouped in 64-token pages ([pages, 64, 576],
-    [pages, 64, 1, 576] or [slots, 576]).  Returns (o bf16 [bs, q_len, h_q, 512],
-    lse fp32 [bs, q_len, h_q])."""
+    """Paged MLA attention.  q bf16 [bs, q_len, h_q, 576], or float8_e4m3fn codes with an
+    float8_e4m3fn cache (the backend's fp8 branch: q quantised with the cache's scale, that
+    scale passed as descale_q and descale_k); k_cache bf16 or float8_e4m3fn with 576-wide
+    token rows grouped in 64-token pages ([pages, 64, 576], [pages, 64, 1, 576] or
+    [slots, 576]).  Returns (o bf16 [bs, q_len, h_q, 512], lse fp32 [bs, q_len, h_q])."""
     _require_cuda(q, k_cache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits,
                   descale_q, descale_k, out, lse, workspace)
-    if q.dim() != 4 or q.dtype != torch.bfloat16 or not q.is_contiguous():
-        raise ValueError("q must be a contiguous bf16 [bs, q_len, h_q, head_dim] tensor")
+    if q.dim() != 4 or q.dtype not in (torch.bfloat16, torch.float8_e4m3fn) or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 or float8_e4m3fn [bs, q_len, h_q, head_dim] tensor")
     bs, q_len, h_q, head_dim = (int(x) for x in q.shape)
     if not k_cache.is_contiguous() or k_cache.shape[-1] != head_dim:
         raise ValueError("k_cache must be contiguous with head_dim-wide rows")
     if k_cache.numel() % (PAGE_SIZE * head_dim):
         raise ValueError("k_cache must hold whole 64-token pages")
     num_pages = k_cache.numel() // (PAGE_SIZE * head_dim)
-    if k_cache.dtype == torch.bfloat16:
-        kv_dtype = DTYPE_BF16
-    elif k_cache.dtype == torch.float8_e4m3fn:
-        kv_dtype = DTYPE_FP8_E4M3
-    else:
+    if k_cache.dtype not in _CACHE_DTYPES:
         raise ValueError(f"unsupported k_cache dtype {k_cache.dtype}")
+    kv_dtype = _CACHE_DTYPES[k_cache.dtype]
     if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.stride(1) != 1:
         raise ValueError("block_table must be a row-major int32 [bs, max_pages] matrix")
     if cache_seqlens.dtype != torch.int32:
@@ -228,11 +279,13 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
         lse = torch.empty((bs, q_len, h_q), dtype=torch.float32, device=dev)
     need = workspace_bytes(bs, q_len, h_q, parts) if bs else 0
     if workspace is None and need:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+        # zero-filled: the leading arrival words must be zero at a workspace's first use
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     sl = cache_seqlens.contiguous()
+    q_dtype = DTYPE_FP8_E4M3 if q.dtype == torch.float8_e4m3fn else DTYPE_BF16
     _check(library().mla_decode_paged(
-        _ptr(q), DTYPE_BF16, bs, q_len, h_q, head_dim, int(head_dim_v), _ptr(k_cache), kv_dtype,
+        _ptr(q), q_dtype, bs, q_len, h_q, head_dim, int(head_dim_v), _ptr(k_cache), kv_dtype,
         num_pages, PAGE_SIZE, _ptr(block_table), block_table.stride(0), int(block_table.shape[1]),
         _ptr(sl), _ptr(tile_scheduler_metadata), parts, _ptr(num_splits), float(softmax_scale),
         int(bool(causal)), _ptr(descale_q), _ptr(descale_k), _ptr(out), _ptr(lse),
@@ -241,6 +294,29 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
 
 
 flash_mla_with_kvcache = mla_decode_paged
+
+
+def set_kv_buffer(k_cache: torch.Tensor, cache_loc: torch.Tensor, k: torch.Tensor,
+                  k_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """token_to_kv_pool.set_kv_buffer for the MLA latent pool: row cache_loc[i] of k_cache
+    ([slots, 576] or any view with 576-wide rows; bf16, float8_e4m3fn or float8_e5m2) receives
+    k[i] (bf16 [n, 576], the latent row whose first 512 columns are the value), an fp8 pool
+    storing k / k_scale rounded to its format.  In place; returns k_cache."""
+    _require_cuda(k_cache, cache_loc, k, k_scale)
+    if k_cache.dtype not in _CACHE_DTYPES or not k_cache.is_contiguous() or k_cache.shape[-1] != 576:
+        raise ValueError("k_cache must be a contiguous bf16 / float8 pool with 576-wide rows")
+    if k.dtype != torch.bfloat16 or k.dim() != 2 or k.shape[1] != 576 or k.stride(1) != 1:
+        raise ValueError("k must be a bf16 [n, 576] matrix with unit column stride")
+    if k_scale is not None and (k_scale.dtype != torch.float32 or k_scale.numel() < 1):
+        raise ValueError("k_scale must be a float32 tensor of one element")
+    loc = cache_loc.contiguous()
+    n = int(k.shape[0])
+    if loc.numel() != n:
+        raise ValueError("one cache_loc entry per token")
+    _check(library().mla_set_kv_buffer(_ptr(k_cache), _CACHE_DTYPES[k_cache.dtype], k_cache.numel() // 576,
+                                       _ptr(loc), _index_dtype(loc), n, _ptr(k), k.stride(0), _ptr(k_scale),
+                                       _stream(k_cache.device)), "mla_set_kv_buffer")
+    return k_cache
 
 
 def read_device_error(device=None) -> int:

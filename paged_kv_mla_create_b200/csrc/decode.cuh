@@ -40,10 +40,20 @@
 //     in tensor memory only when the running maximum grows by more than 2^8, and the
 //     epilogue normalises and writes o and lse.
 //   * A unit whose block range is a whole request writes bf16 o and lse directly; a split
-//     piece writes fp32 partials that combine_splits_kernel merges.
+//     piece writes fp32 partials, then counts its arrival on a per-(request, query tile,
+//     CTA) word of the workspace.  For a request of at most kFusedMergeMaxPieces pieces the
+//     CTA whose arrival completes the count merges the pieces' partials of its 64 rows
+//     (log-sum-exp) once its part is done, with all its warps, and resets the word to zero;
+//     combine_splits_kernel merges requests of more pieces.
+//   * e4m3 queries with an e4m3 cache (the backend page's fp8 recipe: q quantised with the
+//     cache's scale, descale_q and descale_k passed along): S runs as kind::f8f6f4 MMAs (K = 32
+//     per instruction, 18 per tile) straight from the raw page and the e4m3 query rows, both in a
+//     64-byte-swizzled layout (a 64-value row is one swizzle span); only the V chunks each CTA
+//     supplies to PV are widened to f16, after S, by warps 8..11.
 //   * Every wait is bounded (mbar_wait_bounded); out-of-range page ids never fault: TMA
 //     reads zeros for out-of-range coordinates and the error word records the event.
 #pragma once
+#include "combine.cuh"
 #include "ptx.cuh"
 
 namespace mla {
@@ -101,11 +111,18 @@ enum : int {
     kBarOEmpty,                         // leader: 8 softmax warps read O out
     kBarXchg,                           // local (x2): the 128 softmax threads posted row maxima
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
+    kBarPartial,                        // local: the 128 softmax threads stored a split piece
+    kBarVWiden,                         // local, e4m3 q: warps 8..11 read their raw V chunks
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
 };
 
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+// After the barriers: tensor-memory base, abort flag, pending-merge count, and up to two
+// pending merges (request, first split slot, pieces): only a part's first and last units
+// can be pieces of split requests.
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kMaxPendingMerges = 2;
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
 
@@ -113,6 +130,7 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr uint32_t kIdescQK16 = idesc_bf16_f32(128, 128, false, false, true);
 constexpr uint32_t kIdescPV16 = idesc_bf16_f32(128, 256, false, true, true);
+constexpr uint32_t kIdescQK8 = idesc_e4m3_f32(128, 128);
 
 // e4m3 cache: a page (64 rows x 576 one-byte values, 36 KB) lands in the back half of its
 // slot as nine 64 x 64-byte chunks and is widened in place, chunk by chunk from the front,
@@ -122,10 +140,11 @@ constexpr int kPage8Bytes = kPage * kDqk;              // 36 KB
 constexpr int kRaw8Off = kKSlotBytes - kPage8Bytes;    // 36 KB into the slot
 constexpr int kChunk8 = 64 * 64;                       // one 64-row x 64-byte e4m3 chunk
 
-// Widen one e4m3 chunk (64 rows x 64 bytes at src) to f16 (64 rows x 128 bytes at dst,
-// 128-byte swizzle: 16-byte unit u of row t at u ^ (t & 7)).  One warp; the whole chunk
-// is read before any of it is written.
-__device__ __forceinline__ void widen_chunk_e4m3(uint32_t src, uint32_t dst, int lane) {
+// Widen one 8-bit chunk (64 rows x 64 bytes at src; e5m2 when kE5M2, else e4m3) to f16
+// (64 rows x 128 bytes at dst, 128-byte swizzle: 16-byte unit u of row t at u ^ (t & 7)).
+// One warp; the whole chunk is read before any of it is written.
+template <bool kE5M2>
+__device__ __forceinline__ void widen_chunk_fp8(uint32_t src, uint32_t dst, int lane) {
     uint4 v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = ld_shared_v4u(src + 16u * (uint32_t)(lane + 32 * j));
@@ -135,12 +154,41 @@ __device__ __forceinline__ void widen_chunk_e4m3(uint32_t src, uint32_t dst, int
         const int x = lane + 32 * j;        // row x / 4, 16-value quarter x % 4
         const uint32_t t = (uint32_t)(x >> 2), q = (uint32_t)(x & 3);
         const uint32_t row = dst + 128u * t;
-        st_shared_v4u(row + 16u * ((2u * q) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].x), e4m3x2_to_f16x2(v[j].x >> 16),
-                      e4m3x2_to_f16x2(v[j].y), e4m3x2_to_f16x2(v[j].y >> 16));
-        st_shared_v4u(row + 16u * ((2u * q + 1u) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].z),
-                      e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w), e4m3x2_to_f16x2(v[j].w >> 16));
+        st_shared_v4u(row + 16u * ((2u * q) ^ (t & 7u)), fp8x2_to_f16x2<kE5M2>(v[j].x), fp8x2_to_f16x2<kE5M2>(v[j].x >> 16),
+                      fp8x2_to_f16x2<kE5M2>(v[j].y), fp8x2_to_f16x2<kE5M2>(v[j].y >> 16));
+        st_shared_v4u(row + 16u * ((2u * q + 1u) ^ (t & 7u)), fp8x2_to_f16x2<kE5M2>(v[j].z),
+                      fp8x2_to_f16x2<kE5M2>(v[j].z >> 16), fp8x2_to_f16x2<kE5M2>(v[j].w), fp8x2_to_f16x2<kE5M2>(v[j].w >> 16));
     }
     __syncwarp();
+}
+
+// e4m3 queries: Q (64 rows x 576 codes) in shared memory as nine 64 x 64-byte chunks with
+// 64-byte swizzle, and the raw page in the back half of its slot in the same layout.
+constexpr int kQ8Bytes = kChunks * 64 * 64;            // 36 KB
+static_assert(kQ8Bytes <= kQHiBytes, "e4m3 Q fits the Q region");
+
+// Read one raw e4m3 chunk (64 rows x 64 bytes, 64-byte swizzle: 16-byte unit u of row t at
+// u ^ ((t >> 1) & 3)) into registers: lane holds units x = lane + 32 j (row x / 4, unit x % 4).
+__device__ __forceinline__ void load_chunk_sw64(uint32_t src, int lane, uint4 (&v)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t x = (uint32_t)(lane + 32 * j), row = x >> 2, u = x & 3u;
+        v[j] = ld_shared_v4u(src + 64u * row + 16u * (u ^ ((row >> 1) & 3u)));
+    }
+}
+
+// Store the chunk read by load_chunk_sw64 widened to f16 (64 rows x 128 bytes, 128-byte
+// swizzle: unit k of row t at k ^ (t & 7)); e4m3 -> f16 is exact.
+__device__ __forceinline__ void store_chunk_f16(uint32_t dst, int lane, const uint4 (&v)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t x = (uint32_t)(lane + 32 * j), t = x >> 2, u = x & 3u;
+        const uint32_t row = dst + 128u * t;
+        st_shared_v4u(row + 16u * ((2u * u) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].x), e4m3x2_to_f16x2(v[j].x >> 16),
+                      e4m3x2_to_f16x2(v[j].y), e4m3x2_to_f16x2(v[j].y >> 16));
+        st_shared_v4u(row + 16u * ((2u * u + 1u) ^ (t & 7u)), e4m3x2_to_f16x2(v[j].z),
+                      e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w), e4m3x2_to_f16x2(v[j].w >> 16));
+    }
 }
 
 // bf16 pair -> f16 pair (the e4m3 path computes in f16); flags values beyond f16's range.
@@ -169,6 +217,7 @@ struct Params {
     float* lse;                    // [bs, rows]
     float* part_o;                 // [splits, rows, 512]
     float* part_lse;               // [splits, rows]
+    int32_t* arrivals;             // [bs, query tiles, 2]: split pieces arrived (zero between calls)
 };
 
 // The work units of a part, identical in every role: request b, block range [kb0, kb1).
@@ -250,17 +299,23 @@ struct PageWindow {
     }
 };
 
-template <bool kFp8>
+// kKv: the cache's element type, 0 bf16, 1 e4m3, 2 e5m2 (both 8-bit caches are widened to f16
+// for the MMAs); kFp8Q: e4m3 queries (requires an e4m3 cache).
+template <int kKv, bool kFp8Q>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
                   const __grid_constant__ CUtensorMap q_map, const __grid_constant__ Params p) {
+    constexpr bool kFp8 = kKv != 0;
+    constexpr bool kE5M2 = kKv == 2;
+    static_assert(kKv == 1 || !kFp8Q, "e4m3 queries need an e4m3 cache");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pending = reinterpret_cast<int*>(smem + kOffMisc + 8);   // count, then (ub, s0, n) x 2
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -280,7 +335,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_init(bar(kBarKRaw + s), 1);
         }
         // the eight Q warps of the pair, plus the Q TMA's arrival in the bf16 path
-        mbar_init(bar(kBarQFull), (kFp8 ? 0 : 1) + 4);
+        // bf16: the Q TMA + 4 warps' tensor-memory stores; e4m3 cache: the 4 warps; e4m3 q: the TMA
+        mbar_init(bar(kBarQFull), kFp8Q ? 1 : (kFp8 ? 0 : 1) + 4);
+        mbar_init(bar(kBarVWiden), 128);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
@@ -293,7 +350,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         mbar_init(bar(kBarXchg), 128);
         mbar_init(bar(kBarXchg + 1), 128);
         mbar_init(bar(kBarLx), 128);
+        mbar_init(bar(kBarPartial), 128);
         *abort_flag = 0;
+        pending[0] = 0;
         fence_mbarrier_init_cluster();
     }
     if (warp == 1) {
@@ -357,13 +416,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (lane == 0) {
                     ok = mbar_wait_bounded(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, abort_flag);
                     if (ok) {
-                        if constexpr (kFp8) {
+                        if constexpr (kFp8 && !kFp8Q) {
                             mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
                             tma_load_3d_hint(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0, kv_pol);
                         } else {
+                            // the pair's pages complete the leader's barrier: bf16 pages, or raw
+                            // e4m3 pages that S reads as they are (e4m3 queries)
                             const uint32_t kf = bar(kBarKFull + s);
-                            if (leader) mbar_arrive_expect_tx(kf, 2 * kChunks * kBox);
-                            tma_load_3d_pair_hint(slot, &k_map, map_to_cta(kf, 0), 0, row, 0, kv_pol);
+                            if (leader) mbar_arrive_expect_tx(kf, kFp8Q ? 2 * kPage8Bytes : 2 * kChunks * kBox);
+                            tma_load_3d_pair_hint(kFp8Q ? slot + kRaw8Off : slot, &k_map, map_to_cta(kf, 0), 0, row,
+                                                  0, kv_pol);
                         }
                     }
                 }
@@ -371,7 +433,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     alive = false;
                     break;
                 }
-                if constexpr (kFp8) {
+                if constexpr (kFp8 && !kFp8Q) {
                     // the whole warp widens the page in place, then signals the leader
                     const bool landed = mbar_wait_bounded(bar(kBarKRaw + s), (g >> 1) & 1u, abort_flag);
                     if (!__all_sync(0xffffffffu, landed)) {
@@ -380,7 +442,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     }
 #pragma unroll 1
                     for (int c = 0; c < kChunks; ++c)
-                        widen_chunk_e4m3(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
+                        widen_chunk_fp8<kE5M2>(slot + kRaw8Off + c * kChunk8, slot + c * kBox, lane);
                     fence_proxy_async_smem();
                     signal_leader(kBarKFull + s, 8);
                 }
@@ -419,7 +481,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 if (tiles_of(a0, a1) <= 0) continue;
                 if (!first) {
                     tma_prefetch_4d(&q_map, 0, mtile * kRows + kCtaRows * (int32_t)rank, 0, nb);
-                    tma_prefetch_4d(&q_map, 0, mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, nb);
+                    if (!kFp8Q)   // the bf16 view's box is five chunks: two prefetches cover a row
+                        tma_prefetch_4d(&q_map, 0, mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, nb);
                 }
                 first = false;
             }
@@ -433,55 +496,64 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             // ---- Q of the unit
             if (uq > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
             tc_fence_after();
-            if (!kFp8 && quarter == 3 && lane == 0) {
-                if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQHiBytes);
-                tma_load_4d_pair(sbase + kOffQ, &q_map, map_to_cta(bar(kBarQFull), 0), 0,
-                                 mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, ub);
-            }
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)ub * p.rows + rowg) * kDqk);
-            {
-                uint4 v[32];   // the row's columns [0, 256): all loads in flight at once
-#pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = rowg < p.rows ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        w[4 * k] = v[4 * c + k].x;
-                        w[4 * k + 1] = v[4 * c + k].y;
-                        w[4 * k + 2] = v[4 * c + k].z;
-                        w[4 * k + 3] = v[4 * c + k].w;
-                    }
-                    if constexpr (kFp8) {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], q_range);
-                    }
-                    tmem_st16(tmem + lane_off + kTmemQ + 16u * c, w);
+            if constexpr (kFp8Q) {
+                // e4m3 codes of the CTA's 64 rows, all 576 columns: one 36 KB TMA (64-byte swizzle)
+                if (quarter == 3 && lane == 0) {
+                    if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQ8Bytes);
+                    tma_load_4d_pair(sbase + kOffQ, &q_map, map_to_cta(bar(kBarQFull), 0), 0,
+                                     mtile * kRows + kCtaRows * (int32_t)rank, 0, ub);
                 }
-            }
-            if constexpr (kFp8) {
-                // Q columns [256, 576) as f16 into shared memory (128-byte swizzle): lane
-                // quarters 0 / 1 take chunks 0..2 of them, quarters 2 / 3 chunks 3..4
-                const int c0 = quarter < 2 ? 0 : 3, c1 = quarter < 2 ? 3 : kQHiChunks;
-#pragma unroll 1
-                for (int cc = c0; cc < c1; ++cc) {
-                    const uint32_t qrow = sbase + kOffQ + cc * kBox + (uint32_t)rloc * 128u;
-                    uint4 v[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) v[u] = rowg < p.rows ? __ldg(src + 32 + 8 * cc + u) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        st_shared_v4u(qrow + 16u * ((uint32_t)u ^ ((uint32_t)rloc & 7u)),
-                                      bf16x2_to_f16x2(v[u].x, q_range), bf16x2_to_f16x2(v[u].y, q_range),
-                                      bf16x2_to_f16x2(v[u].z, q_range), bf16x2_to_f16x2(v[u].w, q_range));
+            } else {
+                if (!kFp8 && quarter == 3 && lane == 0) {
+                    if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * kQHiBytes);
+                    tma_load_4d_pair(sbase + kOffQ, &q_map, map_to_cta(bar(kBarQFull), 0), 0,
+                                     mtile * kRows + kCtaRows * (int32_t)rank, kQLoChunks, ub);
                 }
-                fence_proxy_async_smem();
-                if (__any_sync(0xffffffffu, q_range) && lane == 0) raise_error(32 /* MLA_DEVERR_Q_RANGE */);
+                const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)ub * p.rows + rowg) * kDqk);
+                {
+                    uint4 v[32];   // the row's columns [0, 256): all loads in flight at once
+    #pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] = rowg < p.rows ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+    #pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w[16];
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            w[4 * k] = v[4 * c + k].x;
+                            w[4 * k + 1] = v[4 * c + k].y;
+                            w[4 * k + 2] = v[4 * c + k].z;
+                            w[4 * k + 3] = v[4 * c + k].w;
+                        }
+                        if constexpr (kFp8) {
+    #pragma unroll
+                            for (int k = 0; k < 16; ++k) w[k] = bf16x2_to_f16x2(w[k], q_range);
+                        }
+                        tmem_st16(tmem + lane_off + kTmemQ + 16u * c, w);
+                    }
+                }
+                if constexpr (kFp8) {
+                    // Q columns [256, 576) as f16 into shared memory (128-byte swizzle): lane
+                    // quarters 0 / 1 take chunks 0..2 of them, quarters 2 / 3 chunks 3..4
+                    const int c0 = quarter < 2 ? 0 : 3, c1 = quarter < 2 ? 3 : kQHiChunks;
+    #pragma unroll 1
+                    for (int cc = c0; cc < c1; ++cc) {
+                        const uint32_t qrow = sbase + kOffQ + cc * kBox + (uint32_t)rloc * 128u;
+                        uint4 v[8];
+    #pragma unroll
+                        for (int u = 0; u < 8; ++u) v[u] = rowg < p.rows ? __ldg(src + 32 + 8 * cc + u) : make_uint4(0, 0, 0, 0);
+    #pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            st_shared_v4u(qrow + 16u * ((uint32_t)u ^ ((uint32_t)rloc & 7u)),
+                                          bf16x2_to_f16x2(v[u].x, q_range), bf16x2_to_f16x2(v[u].y, q_range),
+                                          bf16x2_to_f16x2(v[u].z, q_range), bf16x2_to_f16x2(v[u].w, q_range));
+                    }
+                    fence_proxy_async_smem();
+                    if (__any_sync(0xffffffffu, q_range) && lane == 0) raise_error(32 /* MLA_DEVERR_Q_RANGE */);
+                }
+                tc_wait_st();
+                tc_fence_before();
+                signal_leader(kBarQFull, 9 + quarter);
             }
-            tc_wait_st();
-            tc_fence_before();
-            signal_leader(kBarQFull, 9 + quarter);
             ++uq;
             // ---- partner V of each tile of the unit
             const int32_t* bt_row = p.block_table + (int64_t)ub * p.bt_stride;
@@ -529,24 +601,42 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         alive = false;
                         break;
                     }
+                    if constexpr (kFp8Q) {
+                        // S read the raw page; now this CTA's own V chunks (4n + 2 rank + h, one per
+                        // warp) are widened to f16 into the positions of the same index.  A widened
+                        // chunk (8 KB) can cover raw chunks (4 KB, in the slot's back half) that other
+                        // warps read, and so can the partner chunks stored below: every warp reads its
+                        // raw chunk before any warp writes.
+                        const int oc = 4 * (quarter >> 1) + 2 * (int)rank + (quarter & 1);
+                        uint4 w[8];
+                        load_chunk_sw64(slot + kRaw8Off + oc * kChunk8, lane, w);
+                        mbar_arrive(bar(kBarVWiden));
+                        const bool read_all = mbar_wait_bounded(bar(kBarVWiden), g & 1u, abort_flag);
+                        if (!__all_sync(0xffffffffu, read_all)) {
+                            alive = false;
+                            break;
+                        }
+                        store_chunk_f16(slot + oc * kBox, lane, w);
+                    }
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int x = qt + 128 * j, h = x >> 8, row = (x >> 2) & 63, q4 = x & 3;
                         const int pos = 4 * (h >> 1) + 2 * (1 - (int)rank) + (h & 1);
                         const uint32_t r = slot + pos * kBox + row * 128;
                         const uint32_t sw = (uint32_t)row & 7u;
-                        st_shared_v4u(r + 16u * ((2u * q4) ^ sw), e4m3x2_to_f16x2(v[j].x), e4m3x2_to_f16x2(v[j].x >> 16),
-                                      e4m3x2_to_f16x2(v[j].y), e4m3x2_to_f16x2(v[j].y >> 16));
-                        st_shared_v4u(r + 16u * ((2u * q4 + 1u) ^ sw), e4m3x2_to_f16x2(v[j].z),
-                                      e4m3x2_to_f16x2(v[j].z >> 16), e4m3x2_to_f16x2(v[j].w),
-                                      e4m3x2_to_f16x2(v[j].w >> 16));
+                        st_shared_v4u(r + 16u * ((2u * q4) ^ sw), fp8x2_to_f16x2<kE5M2>(v[j].x),
+                                      fp8x2_to_f16x2<kE5M2>(v[j].x >> 16), fp8x2_to_f16x2<kE5M2>(v[j].y),
+                                      fp8x2_to_f16x2<kE5M2>(v[j].y >> 16));
+                        st_shared_v4u(r + 16u * ((2u * q4 + 1u) ^ sw), fp8x2_to_f16x2<kE5M2>(v[j].z),
+                                      fp8x2_to_f16x2<kE5M2>(v[j].z >> 16), fp8x2_to_f16x2<kE5M2>(v[j].w),
+                                      fp8x2_to_f16x2<kE5M2>(v[j].w >> 16));
                     }
                     fence_proxy_async_smem();
                     signal_leader(kBarVFull + s, 4 + quarter);
                 }
             }
         }
-        if (!kFp8 && quarter == 3 && lane == 0 && *abort_flag) {
+        if ((!kFp8 || kFp8Q) && quarter == 3 && lane == 0 && *abort_flag) {
             // let copies already issued land before shared memory can go away
             const uint64_t t0 = global_timer_ns();
             while (global_timer_ns() - t0 < 200000ull) {
@@ -633,6 +723,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         tc_fence_after();
                         const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
                         const uint32_t d = tmem + kTmemS + 64u * sb;
+                        if constexpr (kFp8Q) {
+                            // e4m3 x e4m3, K = 32: two MMAs per 64-byte chunk
+#pragma unroll
+                            for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+                                for (int kk = 0; kk < 2; ++kk)
+                                    mma_pair_ss_f8(d, smem_desc_sw64(sbase + kOffQ + c * kChunk8 + 32u * kk),
+                                                   smem_desc_sw64(slot + kRaw8Off + c * kChunk8 + 32u * kk),
+                                                   kIdescQK8, (c | kk) ? 1u : 0u);
+                        } else {
 #pragma unroll
                         for (int c = 0; c < kChunks; ++c) {
                             if (c < kQLoChunks) {
@@ -648,6 +748,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                                 smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
                                                 kFp8 ? kIdescQK16 : kIdescQK, 1u);
                             }
+                        }
                         }
                         tc_commit_pair(bar(kBarQKDone + s));
                         tc_commit_pair(bar(kBarSFull + sb));
@@ -695,7 +796,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             if (half == 0) p.lse[(int64_t)b * p.rows + rowg] = -INFINITY;
         };
 
-        uint32_t g = 0, uq = 0;
+        uint32_t g = 0, uq = 0, npartial = 0;
         bool alive = true;
         int ub, kb0, kb1;
         while (alive && iter.next(ub, kb0, kb1)) {
@@ -893,12 +994,54 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 else
                     st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
             }
+            if (!direct && pieces <= kFusedMergeMaxPieces) {
+                // This piece's partial rows are written: make them visible device-wide, then
+                // count the arrival.  The CTA whose arrival completes the count merges them.
+                // (An mbarrier, not bar.sync, gathers the 128 threads: a bounded wait can never
+                // strand them if another role gave up.)
+                __threadfence();
+                mbar_arrive(bar(kBarPartial));
+                if (!mbar_wait_bounded(bar(kBarPartial), npartial & 1u, abort_flag)) break;
+                ++npartial;
+                if (t == 0) {
+                    int32_t* word = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
+                    const int old = atomicAdd(word, 1);
+                    if (old < 0 || old >= pieces) raise_error(128 /* MLA_DEVERR_WORKSPACE_STATE */);
+                    if (old == pieces - 1) {
+                        *word = 0;   // every piece has arrived: ready for the next call
+                        const int k = pending[0];
+                        if (k < kMaxPendingMerges) {
+                            pending[1 + 3 * k] = ub;
+                            pending[2 + 3 * k] = p.num_splits[ub];
+                            pending[3 + 3 * k] = pieces;
+                            pending[0] = k + 1;
+                        } else {
+                            raise_error(8 /* MLA_DEVERR_BAD_METADATA */);
+                        }
+                    }
+                }
+            }
             ++uq;
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    // Merges of the requests whose last piece arrived here, by the whole CTA (the row-max
+    // exchange area is free now and holds the weights).
+    const int npending = pending[0];
+    if (npending > 0 && !*abort_flag) {
+        __threadfence();   // the other pieces' partials: their fences preceded their arrivals
+        const int row_base = mtile * kRows + kCtaRows * (int)rank;
+        const int nrows = min(kCtaRows, p.rows - row_base);
+        for (int k = 0; k < npending && nrows > 0; ++k) {
+            const int mb = pending[1 + 3 * k], s0 = pending[2 + 3 * k], n = pending[3 + 3 * k];
+            merge_rows_cta<kThreads>(p.part_o, p.part_lse, s0, n, p.rows, row_base, nrows,
+                                     p.out + ((int64_t)mb * p.rows + row_base) * kDv,
+                                     p.lse + (int64_t)mb * p.rows + row_base,
+                                     reinterpret_cast<float*>(smem + kOffX), threadIdx.x);
+        }
+    }
     cluster_sync();
     if (warp == 1) {
         tc_fence_after();

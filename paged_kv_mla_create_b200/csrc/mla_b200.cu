@@ -13,6 +13,7 @@
 #include "block_table.cuh"
 #include "combine.cuh"
 #include "decode.cuh"
+#include "kv_write.cuh"
 #include "planner.cuh"
 
 namespace {
@@ -53,18 +54,28 @@ mla_status_t prepare_decode_kernels() {
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
     std::call_once(flags[dev], [dev] {
-        results[dev] = cudaFuncSetAttribute(mla::decode::mla_decode_kernel<false>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            mla::decode::kSmemBytes);
-        if (results[dev] == cudaSuccess)
-            results[dev] = cudaFuncSetAttribute(mla::decode::mla_decode_kernel<true>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                mla::decode::kSmemBytes);
+        const void* kernels[] = {
+            reinterpret_cast<const void*>(mla::decode::mla_decode_kernel<0, false>),
+            reinterpret_cast<const void*>(mla::decode::mla_decode_kernel<1, false>),
+            reinterpret_cast<const void*>(mla::decode::mla_decode_kernel<1, true>),
+            reinterpret_cast<const void*>(mla::decode::mla_decode_kernel<2, false>)};
+        results[dev] = cudaSuccess;
+        for (const void* k : kernels)
+            if (results[dev] == cudaSuccess)
+                results[dev] = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    mla::decode::kSmemBytes);
     });
     return from_cuda(results[dev]);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout: arrival words int32 [bs, query tiles, 2], then the split partials
+// fp32 [splits, rows, 512] and their lse fp32 [splits, rows], each 256-byte aligned.
+size_t arrival_bytes(int32_t bs, int32_t q_len, int32_t h_q) {
+    const size_t tiles = ((size_t)q_len * (size_t)h_q + 127) / 128;
+    return align256((size_t)bs * tiles * 2 * sizeof(int32_t));
+}
 
 }  // namespace
 
@@ -138,11 +149,51 @@ mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
     return from_cuda(cudaGetLastError());
 }
 
+mla_status_t mla_build_decode_metadata(
+    const int32_t* req_to_token, int64_t req_to_token_rows, int64_t req_to_token_stride,
+    const void* req_pool_indices, int32_t rpi_dtype, const void* seq_lens, int32_t seq_lens_dtype,
+    int32_t seq_len_add, int32_t bs, int32_t* block_table, int64_t block_table_stride,
+    int32_t max_pages, int32_t page_size, int32_t fill_tail, int32_t num_heads_per_head_k,
+    int32_t num_heads_k, int32_t is_fp8_kvcache, int32_t sm_count, int32_t* cache_seqlens,
+    int32_t* tile_scheduler_metadata, int32_t* num_splits, mla_stream_t stream) {
+    (void)is_fp8_kvcache;  // accepted for call compatibility; the plan does not depend on it
+    const int32_t parts = mla_num_sm_parts(sm_count, num_heads_per_head_k, num_heads_k);
+    if (bs < 0 || max_pages < 0 || page_size != 64 || parts < 1 || bs > (1 << 20))
+        return MLA_ERR_INVALID_ARG;
+    if (rpi_dtype != MLA_DTYPE_INT32 && rpi_dtype != MLA_DTYPE_INT64) return MLA_ERR_INVALID_ARG;
+    if (seq_lens_dtype != MLA_DTYPE_INT32 && seq_lens_dtype != MLA_DTYPE_INT64)
+        return MLA_ERR_INVALID_ARG;
+    if (!tile_scheduler_metadata || !num_splits || !is_aligned(tile_scheduler_metadata, 16))
+        return MLA_ERR_INVALID_ARG;
+    if (bs > 0 && (!req_to_token || !req_pool_indices || !seq_lens || !block_table))
+        return MLA_ERR_INVALID_ARG;
+    if (bs > 0 && (req_to_token_rows <= 0 || req_to_token_stride <= 0 || block_table_stride < max_pages))
+        return MLA_ERR_INVALID_ARG;
+    const int64_t entries = (int64_t)bs * max_pages;
+    const int64_t table_ctas = (entries + mla::kPlannerThreads - 1) / mla::kPlannerThreads;
+    if (table_ctas + 1 > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)(1 + table_ctas));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define MLA_MD_LAUNCH(IT, LT)                                                                      \
+    mla::decode_metadata_kernel<IT, LT><<<grid, mla::kPlannerThreads, 0, st>>>(                   \
+        req_to_token, req_to_token_rows, req_to_token_stride,                                      \
+        static_cast<const IT*>(req_pool_indices), static_cast<const LT*>(seq_lens), seq_len_add,  \
+        bs, block_table, block_table_stride, max_pages, fill_tail, parts, cache_seqlens,           \
+        tile_scheduler_metadata, num_splits)
+    if (rpi_dtype == MLA_DTYPE_INT64 && seq_lens_dtype == MLA_DTYPE_INT64) MLA_MD_LAUNCH(int64_t, int64_t);
+    else if (rpi_dtype == MLA_DTYPE_INT64) MLA_MD_LAUNCH(int64_t, int32_t);
+    else if (seq_lens_dtype == MLA_DTYPE_INT64) MLA_MD_LAUNCH(int32_t, int64_t);
+    else MLA_MD_LAUNCH(int32_t, int32_t);
+#undef MLA_MD_LAUNCH
+    return from_cuda(cudaGetLastError());
+}
+
 size_t mla_decode_workspace_bytes(int32_t bs, int32_t q_len, int32_t h_q, int32_t num_sm_parts) {
     if (bs <= 0 || q_len <= 0 || h_q <= 0 || num_sm_parts <= 0) return 0;
     const size_t splits = (size_t)bs + (size_t)num_sm_parts;
     const size_t rows = (size_t)q_len * (size_t)h_q;
-    return align256(splits * rows * 512 * sizeof(float)) + align256(splits * rows * sizeof(float));
+    return arrival_bytes(bs, q_len, h_q) + align256(splits * rows * 512 * sizeof(float)) +
+           align256(splits * rows * sizeof(float));
 }
 
 mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_t q_len,
@@ -157,8 +208,11 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
                               mla_stream_t stream) {
     if (bs < 0 || q_len <= 0 || h_q <= 0 || num_sm_parts < 1) return MLA_ERR_INVALID_ARG;
     if (head_dim != 576 || head_dim_v != 512 || page_size != 64) return MLA_ERR_UNSUPPORTED;
-    if (q_dtype != MLA_DTYPE_BF16) return MLA_ERR_UNSUPPORTED;
-    if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+    if (q_dtype != MLA_DTYPE_BF16 && q_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+    if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3 && kv_dtype != MLA_DTYPE_FP8_E5M2)
+        return MLA_ERR_INVALID_ARG;
+    // e4m3 queries run e4m3 x e4m3 MMAs: only with an e4m3 cache (the backend's fp8 branch)
+    if (q_dtype == MLA_DTYPE_FP8_E4M3 && kv_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
     if (kv_dtype == MLA_DTYPE_BF16 && descale_k) return MLA_ERR_INVALID_ARG;  // fp8 caches only
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
@@ -195,7 +249,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     std::memset(&v_map, 0, sizeof v_map);
     std::memset(&q_map, 0, sizeof q_map);
     const cuuint64_t pool_rows = (cuuint64_t)num_pages * 64;
-    const bool fp8 = kv_dtype == MLA_DTYPE_FP8_E4M3;
+    const bool fp8 = kv_dtype != MLA_DTYPE_BF16;
     if (!fp8) {
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {1152, 128};
@@ -211,19 +265,33 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MLA_ERR_CUDA;
     } else {
-        // e4m3: (64 one-byte columns, pool rows [576 B], 9 column chunks [64 B]), no swizzle;
-        // a K load = one page as 9 chunks of 64 rows x 64 bytes (36 KB), a V load = 2 chunks.
+        // 8-bit: (64 one-byte columns, pool rows [576 B], 9 column chunks [64 B]); a K load = one
+        // page as 9 chunks of 64 rows x 64 bytes (36 KB).  Unswizzled for bf16 queries (the page
+        // is widened to f16 before S); 64-byte swizzle for e4m3 queries (S reads it as it is).
+        const bool q8 = q_dtype == MLA_DTYPE_FP8_E4M3;
         const cuuint64_t gdim[3] = {64, pool_rows, 9};
         const cuuint64_t gstride[2] = {576, 64};
         const cuuint32_t kbox[3] = {64, 64, 9};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&k_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(k_cache), gdim, gstride,
-                   kbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   kbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   q8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MLA_ERR_CUDA;
         v_map = k_map;   // the e4m3 path reads partner V through registers
     }
-    {
+    if (q_dtype == MLA_DTYPE_FP8_E4M3) {
+        // e4m3 q: (64 one-byte columns, rows of a request [576 B], 9 column chunks [64 B],
+        // requests); a load = 64 query rows x all 576 columns (36 KB), 64-byte swizzle
+        const cuuint64_t gdim[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)bs};
+        const cuuint64_t gstride[3] = {576, 64, (cuuint64_t)rows * 576};
+        const cuuint32_t box[4] = {64, 64, 9, 1};
+        const cuuint32_t estride[4] = {1, 1, 1, 1};
+        if (encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(q), gdim, gstride, box,
+                   estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    } else {
         const cuuint64_t gdim[4] = {64, (cuuint64_t)rows, 9, (cuuint64_t)bs};
         const cuuint64_t gstride[3] = {1152, 128, (cuuint64_t)rows * 1152};
         const cuuint32_t box[4] = {64, 64, 5, 1};
@@ -255,23 +323,60 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     p.causal = causal;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
-    p.part_o = static_cast<float*>(workspace);
-    p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.arrivals = reinterpret_cast<int32_t*>(ws);
+    p.part_o = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q));
+    p.part_lse = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q) +
                                           align256(splits * rows * 512 * sizeof(float)));
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
-    if (fp8)
-        mla::decode::mla_decode_kernel<true><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
-            k_map, v_map, q_map, p);
+    using mla::decode::kSmemBytes;
+    using mla::decode::kThreads;
+    if (q_dtype == MLA_DTYPE_FP8_E4M3)
+        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+    else if (kv_dtype == MLA_DTYPE_FP8_E4M3)
+        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+    else if (kv_dtype == MLA_DTYPE_FP8_E5M2)
+        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
     else
-        mla::decode::mla_decode_kernel<false><<<grid, mla::decode::kThreads, mla::decode::kSmemBytes, s>>>(
-            k_map, v_map, q_map, p);
+        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     const dim3 cgrid((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
     mla::combine_splits_kernel<<<cgrid, mla::kCombineWarps * 32, 0, s>>>(
         p.part_o, p.part_lse, num_splits, rows, p.out, lse);
+    return from_cuda(cudaGetLastError());
+}
+
+mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slots, const void* cache_loc,
+                               int32_t loc_dtype, int32_t n_tokens, const void* k, int64_t k_row_stride,
+                               const float* k_scale, mla_stream_t stream) {
+    if (n_tokens < 0 || num_slots < 0) return MLA_ERR_INVALID_ARG;
+    if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3 && kv_dtype != MLA_DTYPE_FP8_E5M2)
+        return MLA_ERR_INVALID_ARG;
+    if (loc_dtype != MLA_DTYPE_INT32 && loc_dtype != MLA_DTYPE_INT64) return MLA_ERR_INVALID_ARG;
+    if (kv_dtype == MLA_DTYPE_BF16 && k_scale) return MLA_ERR_INVALID_ARG;   // a scale is for fp8 pools
+    if (n_tokens == 0) return MLA_OK;
+    if (!kv_cache || !cache_loc || !k) return MLA_ERR_INVALID_ARG;
+    if (k_row_stride < 576 || k_row_stride % 8 != 0 || !is_aligned(k, 16)) return MLA_ERR_INVALID_ARG;
+    if (!is_aligned(kv_cache, kv_dtype == MLA_DTYPE_BF16 ? 16 : 8)) return MLA_ERR_INVALID_ARG;
+    const dim3 grid((unsigned)((n_tokens + mla::kKvWriteWarps - 1) / mla::kKvWriteWarps));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* pool = static_cast<uint8_t*>(kv_cache);
+    const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(k);
+#define MLA_KV_LAUNCH(FMT, LT)                                                                     \
+    mla::set_kv_buffer_kernel<FMT, LT><<<grid, mla::kKvWriteWarps * 32, 0, st>>>(                  \
+        pool, num_slots, static_cast<const LT*>(cache_loc), n_tokens, kk, k_row_stride, k_scale)
+    const bool l64 = loc_dtype == MLA_DTYPE_INT64;
+    if (kv_dtype == MLA_DTYPE_BF16) {
+        if (l64) MLA_KV_LAUNCH(0, int64_t); else MLA_KV_LAUNCH(0, int32_t);
+    } else if (kv_dtype == MLA_DTYPE_FP8_E4M3) {
+        if (l64) MLA_KV_LAUNCH(1, int64_t); else MLA_KV_LAUNCH(1, int32_t);
+    } else {
+        if (l64) MLA_KV_LAUNCH(2, int64_t); else MLA_KV_LAUNCH(2, int32_t);
+    }
+#undef MLA_KV_LAUNCH
     return from_cuda(cudaGetLastError());
 }
 
@@ -336,6 +441,12 @@ extern "C" mla_status_t mla_decode_paged_noalloc(
     if (bs > 0) {
         const mla_status_t st = noalloc_scratch_address(&scratch);
         if (st != MLA_OK) return st;
+        // The array keeps whatever the last call left; its leading arrival words must be zero
+        // when the attention starts (a completed call leaves them zero, an aborted one may not).
+        if (q_len > 0 && h_q > 0 &&
+            cudaMemsetAsync(scratch, 0, arrival_bytes(bs, q_len, h_q), reinterpret_cast<cudaStream_t>(stream)) !=
+                cudaSuccess)
+            return MLA_ERR_CUDA;
     }
     return mla_decode_paged(q, q_dtype, bs, q_len, h_q, head_dim, head_dim_v, k_cache, kv_dtype,
                             num_pages, page_size, block_table, block_table_stride, max_pages,

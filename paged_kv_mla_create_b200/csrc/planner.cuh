@@ -13,8 +13,8 @@
 // part i's budget left, either it fits (r >= blocks + F), or, after skipping to a fresh
 // part when r <= F, its first piece takes r - F blocks, the following parts take
 // Q = P - F blocks each, and the last piece takes the rest (1..Q blocks) -- a closed form
-// with one division.  One thread runs that O(bs) recurrence (each step a few
-// instructions, so a request costs what one part's step cost before); then one thread
+// whose one division is needed only when a request spans more than one further part.  One
+// thread runs that O(bs) recurrence, a short chain of compares per request; then one thread
 // per part reads its row off the per-request results by binary search: its first piece
 // belongs to the first request whose last part is >= i, its last to the last request
 // whose first part is <= i.  Batches larger than kPlannerSmemLens take the part-by-part
@@ -40,19 +40,33 @@ __device__ __forceinline__ int div_small(int a, int q, float q_inv) {
     return m;
 }
 
-__global__ void __launch_bounds__(kPlannerThreads)
-get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, int32_t parts,
-                        int32_t* __restrict__ md, int32_t* __restrict__ num_splits) {
-    __shared__ int32_t s_nb[kPlannerSmemLens + 1];   // blocks of request b
-    __shared__ int32_t s_fp[kPlannerSmemLens];       // first part of request b
-    __shared__ int32_t s_lp[kPlannerSmemLens];       // last part of request b
-    __shared__ int32_t s_x0[kPlannerSmemLens];       // blocks of its first piece
-    __shared__ int32_t s_cum[kPlannerSmemLens];      // num_splits[b + 1]
-    __shared__ long long s_warp_sum[kPlannerThreads / 32];
+struct PlannerSmem {
+    int32_t nb[kPlannerSmemLens + 1];   // blocks of request b
+    int32_t fp[kPlannerSmemLens];       // first part of request b
+    int32_t lp[kPlannerSmemLens];       // last part of request b
+    int32_t x0[kPlannerSmemLens];       // blocks of its first piece
+    int32_t cum[kPlannerSmemLens];      // num_splits[b + 1]
+    long long warp_sum[kPlannerThreads / 32];
+};
+
+// The plan, computed by one CTA of kPlannerThreads threads.  len_of(b) is request b's KV
+// length (read once per request, by the first loop); cache_seqlens_out, when not null,
+// receives those lengths as int32.
+template <typename LenFn>
+__device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t parts,
+                                           int32_t* __restrict__ md, int32_t* __restrict__ num_splits,
+                                           int32_t* __restrict__ cache_seqlens_out, PlannerSmem& sm) {
+    int32_t* s_nb = sm.nb;
+    int32_t* s_fp = sm.fp;
+    int32_t* s_lp = sm.lp;
+    int32_t* s_x0 = sm.x0;
+    int32_t* s_cum = sm.cum;
+    long long* s_warp_sum = sm.warp_sum;
     const bool staged = bs <= kPlannerSmemLens;
     long long local = 0;
     for (int b = threadIdx.x; b < bs; b += blockDim.x) {
-        const int32_t L = cache_seqlens[b];
+        const int32_t L = len_of(b);
+        if (cache_seqlens_out) cache_seqlens_out[b] = L;
         const int32_t nb = L > 0 ? (L + 63) / 64 : 0;
         if (staged) s_nb[b] = nb;
         local += nb + kFixedOverhead;
@@ -74,7 +88,7 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
         if (threadIdx.x == 0) {
             auto blocks_of = [&](int b) -> int {
                 if (b >= bs) return 0;
-                const int32_t L = cache_seqlens[b];
+                const int32_t L = len_of(b);
                 return L > 0 ? (L + 63) / 64 : 0;
             };
             num_splits[0] = 0;
@@ -110,27 +124,35 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
     }
 
     if (threadIdx.x == 0) {
-        // Straight-line step: both outcomes (the request fits / it is split) are computed and
-        // one is selected, so an iteration is one short dependency chain through r and i.
+        // The walk's loop-carried state is (i, r): the part and what is left of its budget.
+        // Entering request b of c = blocks + F: a part with r <= F and r < c ends unused; the
+        // request then fits (r >= c) or is split: its first piece takes r - F blocks, m full
+        // middle parts take Q blocks each and the last piece the rest, last = rem - m Q with
+        // rem = c - r, leaving Q - last.  m > 0 only when rem - 1 >= Q, so the division stays
+        // off the common path.
         int i = 0, r = P, cum = 0;
         int nb = s_nb[0];
         for (int b = 0; b < bs; ++b) {
             const int nb_next = s_nb[b + 1];
             const int c = nb + kFixedOverhead;
-            const bool skip = (r < c) & (r <= kFixedOverhead);   // the part ends with budget unused
-            r = skip ? P : r;
-            i += skip ? 1 : 0;
-            const bool fits = r >= c;
-            const int x0s = r - kFixedOverhead;                   // split: 1 <= x0s < nb
-            const int rem = nb - x0s;                             // split: >= 1
-            const int m = div_small(max(rem - 1, 0), Q, qinv);    // split: full middle pieces
-            const int last = rem - m * Q;                         // split: 1..Q
+            if (r < c && r <= kFixedOverhead) {
+                r = P;
+                ++i;
+            }
             s_fp[b] = i;
-            i = fits ? i : i + 1 + m;
-            r = fits ? r - c : P - last - kFixedOverhead;
+            if (r >= c) {
+                r -= c;
+                s_x0[b] = nb;
+                cum += 1;
+            } else {
+                const int rem = c - r;                                   // >= 1
+                const int m = rem - 1 >= Q ? div_small(rem - 1, Q, qinv) : 0;
+                s_x0[b] = r - kFixedOverhead;                            // 1 <= x0 < nb
+                i += 1 + m;
+                r = Q - (rem - m * Q);
+                cum += 2 + m;
+            }
             s_lp[b] = i;
-            s_x0[b] = fits ? nb : x0s;
-            cum += fits ? 1 : 2 + m;
             s_cum[b] = cum;
             nb = nb_next;
         }
@@ -176,6 +198,13 @@ get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, i
         row[0] = r0;
         row[1] = r1;
     }
+}
+
+__global__ void __launch_bounds__(kPlannerThreads)
+get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, int32_t parts,
+                        int32_t* __restrict__ md, int32_t* __restrict__ num_splits) {
+    __shared__ PlannerSmem sm;
+    plan_parts([&](int b) -> int32_t { return cache_seqlens[b]; }, bs, parts, md, num_splits, nullptr, sm);
 }
 
 }  // namespace mla

@@ -148,11 +148,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
            | ((uint32_t)(M >> 4) << 24);          // M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4 with e4m3 A and B (K-major) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4)                              // D format: f32
+           | (0u << 7) | (0u << 10)               // A, B format: e4m3
+           | ((uint32_t)(N >> 3) << 17)           // N / 8
+           | ((uint32_t)(M >> 4) << 24);          // M / 16
+}
+
 // Shared-memory matrix descriptor (sm_100 format, version 1), 128-byte swizzle.
 // lbo / sbo in bytes.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// As smem_desc_sw128 for a K-major operand with 64-byte rows and 64-byte swizzle (8-row
+// groups 512 bytes apart): an e4m3 tile whose 64-value rows are one swizzle span.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(512 >> 4) << 32) |
+           (1ull << 46) | (4ull << 61);
 }
 
 // 32 lanes x 32-bit: thread t of the warp reads lane (base lane + t), N consecutive columns.
@@ -282,8 +297,16 @@ __device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
-// Arrive on `bar` (same offset) in both CTAs of the pair once the pair MMAs issued so far
-// have completed.
+// As mma_pair_ss for kind::f8f6f4 (8-bit A and B, K = 32 per instruction).
+__device__ __forceinline__ void mma_pair_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // As mma_pair_ss with A read from tensor memory: each CTA's 64 rows of A in lanes 0..63
 // at columns a_tmem.., two bf16 of consecutive k per 32-bit column.
 __device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -295,6 +318,8 @@ __device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// Arrive on `bar` (same offset) in both CTAs of the pair once the pair MMAs issued so far
+// have completed.
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
@@ -323,6 +348,24 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
     const uint16_t v = (uint16_t)two_bytes;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
     return r;
+}
+
+// Two e5m2 values (first in the low byte) -> two f16 (first in the low half); exact (e5m2 is
+// f16 with its low mantissa byte dropped).
+__device__ __forceinline__ uint32_t e5m2x2_to_f16x2(uint32_t two_bytes) {
+    uint32_t r;
+    const uint16_t v = (uint16_t)two_bytes;
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+// Two 8-bit cache values -> two f16: e5m2 (kE5M2) or e4m3.
+template <bool kE5M2>
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two_bytes) {
+    if constexpr (kE5M2)
+        return e5m2x2_to_f16x2(two_bytes);
+    else
+        return e4m3x2_to_f16x2(two_bytes);
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4u(uint32_t addr) {

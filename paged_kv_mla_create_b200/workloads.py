@@ -34,12 +34,13 @@ D_V = 512
 SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
 POISON = 3.0e4          # finite poison for unused pages / tail rows (bf16 rounds it to 29952)
 POISON_FP8 = 448.0      # largest finite e4m3 value
+POISON_E5M2 = 57344.0   # largest finite e5m2 value
 
 
 @dataclasses.dataclass
 class Workload:
     name: str
-    q: torch.Tensor                 # bf16 [bs, q_len, h, 576]
+    q: torch.Tensor                 # bf16, or e4m3 codes, [bs, q_len, h, 576]
     kv_cache: torch.Tensor          # bf16 or float8_e4m3fn [num_pages, 64, 576]
     req_to_token: torch.Tensor      # int32 [bs + 3, max_ctx]
     req_pool_indices: torch.Tensor  # int64 [bs]
@@ -48,7 +49,7 @@ class Workload:
     num_draft_tokens: int           # 0 in decode, q_len in target-verify
     softmax_scale: float
     causal: bool
-    descale_q: Optional[torch.Tensor]  # fp32 [1] (fp8 cache only)
+    descale_q: Optional[torch.Tensor]  # fp32 [1] (fp8 cache only): the scale q was quantised with
     descale_k: Optional[torch.Tensor]  # fp32 [1] (fp8 cache only)
 
     @property
@@ -65,7 +66,11 @@ class Workload:
 
     @property
     def is_fp8(self) -> bool:
-        return self.kv_cache.dtype == torch.float8_e4m3fn
+        return self.kv_cache.dtype in (torch.float8_e4m3fn, torch.float8_e5m2)
+
+    @property
+    def q_is_fp8(self) -> bool:
+        return self.q.dtype == torch.float8_e4m3fn
 
     @property
     def max_pages(self) -> int:
@@ -110,9 +115,12 @@ def _draw_lengths(rng: np.random.Generator, recipe, bs: int) -> List[int]:
 def make_case(seq_lens: List[int], h: int, q_len: int = 1, kv: str = "bf16",
               verify: bool = False, seed: int = 0, poison: bool = False,
               pool_pages: Optional[int] = None, name: str = "custom",
-              pool_factor: float = 1.25) -> Workload:
+              pool_factor: float = 1.25, q_fp8: bool = False) -> Workload:
     """Draw one workload.  seq_lens are prefix lengths; in target-verify each request
-    gets q_len more positions (the draft tokens) before attention."""
+    gets q_len more positions (the draft tokens) before attention.  With an fp8 cache,
+    q_fp8 hands q over as e4m3 codes the way the FlashMLA backend page's fp8 branch does:
+    quantised with the cache's own scale (q_scale = k_scale), saturating at +-448, with
+    descale_q = that scale."""
     rng = np.random.default_rng(seed)
     bs = len(seq_lens)
     n_draft = q_len if verify else 0
@@ -151,24 +159,32 @@ def make_case(seq_lens: List[int], h: int, q_len: int = 1, kv: str = "bf16",
                 marks[owned[b][-1], tail:] = True
         signs = np.where(rng.random((int(marks.sum()), D_QK)) < 0.5, -1.0, 1.0)
         x[marks] = 0.0
+    if q_fp8 and kv != "fp8":
+        raise ValueError("e4m3 queries go with an e4m3 cache")
     if kv == "bf16":
         if poison:
             x[marks] = (signs * POISON).astype(np.float32)
         kv_cache = torch.from_numpy(x).to(torch.bfloat16)
-    elif kv == "fp8":
+    elif kv in ("fp8", "e5m2"):
+        # per-tensor scale: the largest magnitude maps to the format's largest finite value
+        top = POISON_FP8 if kv == "fp8" else POISON_E5M2
         amax = float(np.abs(x).max()) if x.size else 0.0
-        scale = np.float32(amax / 448.0) if amax > 0 else np.float32(1.0)
+        scale = np.float32(amax / top) if amax > 0 else np.float32(1.0)
         y = (x / scale).astype(np.float32)
         if poison:
-            y[marks] = (signs * POISON_FP8).astype(np.float32)
-        kv_cache = torch.from_numpy(y).to(torch.float8_e4m3fn)
+            y[marks] = (signs * top).astype(np.float32)
+        kv_cache = torch.from_numpy(y).to(torch.float8_e4m3fn if kv == "fp8" else torch.float8_e5m2)
         descale_k = torch.tensor([float(scale)], dtype=torch.float32)
         descale_q = torch.ones(1, dtype=torch.float32)
+        if q_fp8:
+            qb = q.to(torch.bfloat16).float()
+            q = (qb / float(scale)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+            descale_q = torch.tensor([float(scale)], dtype=torch.float32)
     else:
         raise ValueError(kv)
     return Workload(
         name=name,
-        q=q.to(torch.bfloat16),
+        q=q if q.dtype == torch.float8_e4m3fn else q.to(torch.bfloat16),
         kv_cache=kv_cache,
         req_to_token=torch.from_numpy(req_to_token),
         req_pool_indices=torch.from_numpy(rpi),
@@ -182,12 +198,14 @@ def make_case(seq_lens: List[int], h: int, q_len: int = 1, kv: str = "bf16",
     )
 
 
-def make_workload(index: int, poison: bool = False, seed: Optional[int] = None) -> Workload:
-    """One of the five configured workloads, seeded with 1000 + index."""
+def make_workload(index: int, poison: bool = False, seed: Optional[int] = None,
+                  q_fp8: bool = False) -> Workload:
+    """One of the five configured workloads, seeded with 1000 + index (q_fp8: its queries as
+    e4m3 codes, for the fp8-cache workload)."""
     cfg = CONFIGS[index]
     s = 1000 + index if seed is None else seed
     rng = np.random.default_rng(s)
     lengths = _draw_lengths(rng, cfg["lengths"], cfg["bs"])
     return make_case(lengths, cfg["h"], cfg["q_len"], cfg["kv"], cfg.get("verify", False),
                      seed=s + 7919, poison=poison, pool_pages=cfg.get("pool_pages"),
-                     name=cfg["name"])
+                     name=cfg["name"] + (", e4m3 q" if q_fp8 else ""), q_fp8=q_fp8)

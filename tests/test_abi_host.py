@@ -51,8 +51,12 @@ def test_workspace_bytes():
     lib = mla.library()
     ws = lib.mla_decode_workspace_bytes(64, 1, 128, 74)
     rows, splits = 128, 64 + 74
-    expect = -(-splits * rows * 512 * 4 // 256) * 256 + -(-splits * rows * 4 // 256) * 256
+    a256 = lambda x: -(-x // 256) * 256
+    # arrival words [bs, query tiles, 2] int32, then the partials and their lse
+    expect = a256(64 * 1 * 2 * 4) + a256(splits * rows * 512 * 4) + a256(splits * rows * 4)
     assert ws == expect
+    ws4 = lib.mla_decode_workspace_bytes(32, 4, 128, 18)
+    assert ws4 == a256(32 * 4 * 2 * 4) + a256(50 * 512 * 512 * 4) + a256(50 * 512 * 4)
     assert lib.mla_decode_workspace_bytes(0, 1, 128, 74) == 0
     assert lib.mla_decode_workspace_bytes(1, 1, 128, 0) == 0
 
@@ -73,7 +77,9 @@ def test_decode_validation_happens_before_any_launch():
     assert _decode(lib, head_dim=512) == 2               # unsupported head dims
     assert _decode(lib, head_dim_v=576) == 2
     assert _decode(lib, page_size=32) == 2
-    assert _decode(lib, q_dtype=1) == 2                  # fp8 q: not implemented
+    assert _decode(lib, q_dtype=1) == 2                  # e4m3 q needs an e4m3 cache
+    assert _decode(lib, q_dtype=1, kv_dtype=4) == 2      # ... not e5m2
+    assert _decode(lib, q_dtype=3) == 1                  # not a query type
     assert _decode(lib, kv_dtype=7) == 1
     assert _decode(lib, causal=2) == 1
     assert _decode(lib, q=None) == 1
@@ -86,6 +92,22 @@ def test_decode_validation_happens_before_any_launch():
     assert _decode(lib, scale=float("nan")) == 1
     assert _decode(lib, dk=1 << 29) == 1                 # descale_k with a bf16 cache
     assert _decode(lib, q_len=1, h_q=65535 * 128 + 1) == 2   # more query tiles than grid.y holds
+
+
+def test_set_kv_buffer_validation():
+    lib = mla.library()
+    kv = lib.mla_set_kv_buffer
+    ok = dict(pool=1 << 20, dt=1, slots=100, loc=1 << 21, loc_dt=3, n=4, k=1 << 22, stride=576,
+              scale=None, stream=None)
+    assert kv(*{**ok, "n": 0}.values()) == 0                 # nothing to write
+    assert kv(*{**ok, "dt": 9}.values()) == 1
+    assert kv(*{**ok, "loc_dt": 0}.values()) == 1
+    assert kv(*{**ok, "dt": 0, "scale": 1 << 23}.values()) == 1   # a scale is for fp8 pools
+    assert kv(*{**ok, "stride": 570}.values()) == 1
+    assert kv(*{**ok, "stride": 580}.values()) == 1          # not a multiple of 8
+    assert kv(*{**ok, "k": (1 << 22) + 8}.values()) == 1     # misaligned k
+    assert kv(*{**ok, "pool": None}.values()) == 1
+    assert kv(*{**ok, "n": -1}.values()) == 1
 
 
 def test_block_table_and_planner_validation():
@@ -106,3 +128,14 @@ def test_block_table_and_planner_validation():
     assert md(1 << 20, -1, 128, 1, 0, 148, 1 << 21, 1 << 22, None) == 1
     assert md(1 << 20, 2, 128, 1, 0, 148, (1 << 21) + 4, 1 << 22, None) == 1   # misaligned rows
     assert md(1 << 20, 2, 128, 1, 0, 148, None, 1 << 22, None) == 1
+    dm = lib.mla_build_decode_metadata
+    okm = dict(r2t=1 << 20, rows=5, stride=192, rpi=1 << 21, rpi_dt=3, sl=1 << 22, sl_dt=2, add=0,
+               bs=2, out=1 << 23, out_stride=3, max_pages=3, page=64, fill=1, heads=128, hk=1,
+               fp8=0, sms=148, cl=None, md=1 << 24, ns=1 << 25, stream=None)
+    assert dm(*{**okm, "page": 32}.values()) == 1
+    assert dm(*{**okm, "sms": 0}.values()) == 1
+    assert dm(*{**okm, "heads": 0}.values()) == 1
+    assert dm(*{**okm, "sl_dt": 0}.values()) == 1
+    assert dm(*{**okm, "md": (1 << 24) + 4}.values()) == 1
+    assert dm(*{**okm, "r2t": None}.values()) == 1
+    assert dm(*{**okm, "out_stride": 2}.values()) == 1

@@ -1,8 +1,8 @@
 """Parity of the CUDA path (through the C ABI) with the CPU fp64 oracle.
 
 Page table and split plan: bit-exact.  Attention: max-abs 2e-2 and relative-L2 5e-3 on
-o and on lse (fp8 caches are compared with the oracle run on the same e4m3 codes and
-descale, i.e. on the dequantised cache).  Small cases are compared element by element;
+o and on lse (fp8 caches, and e4m3 queries, are compared with the oracle run on the same
+e4m3 codes and descales, i.e. on the dequantised values).  Small cases are compared element by element;
 the five full-size workloads, in the launch configuration the benchmark times, are
 compared on sampled rows that the oracle computes one by one."""
 import math
@@ -48,7 +48,8 @@ def oracle_rows(wl, rows):
         wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices, wl.cache_seqlens, rows,
         wl.softmax_scale, wl.causal, kv_is_fp8=wl.is_fp8,
         descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
-        descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+        descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0,
+        q_is_fp8=wl.q_is_fp8)
 
 
 def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
@@ -87,7 +88,8 @@ def check_full(mla, wl, parts=None):
                                        wl.cache_seqlens, wl.softmax_scale, wl.causal,
                                        kv_is_fp8=wl.is_fp8,
                                        descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
-                                       descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+                                       descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0,
+                                       q_is_fp8=wl.q_is_fp8)
     assert_close(o, lse, ref_o, ref_lse, wl.name)
     assert mla.read_device_error() == 0
 
@@ -138,6 +140,21 @@ def test_fp8_cache(mla, lens, h, q_len):
                                 poison=True))
 
 
+@pytest.mark.parametrize("lens,h,q_len", [([37, 130], 16, 1), ([1, 63, 64, 65, 127, 128, 129], 128, 1),
+                                         ([1000, 62, 129, 1], 128, 4), ([300, 5000], 40, 3)])
+def test_fp8_queries(mla, lens, h, q_len):
+    """e4m3 queries against an e4m3 cache (the backend page's fp8 branch: q quantised with the
+    cache's scale): S on e4m3 x e4m3 tensor cores; the oracle runs on the same codes."""
+    check_full(mla, W.make_case(lens, h=h, q_len=q_len, kv="fp8", verify=q_len > 1, seed=51,
+                                poison=True, q_fp8=True))
+
+
+@pytest.mark.parametrize("parts", [2, 7, 74])
+def test_fp8_queries_forced_splits(mla, parts):
+    check_full(mla, W.make_case([2000, 33, 700, 4000, 129], h=128, kv="fp8", seed=52, poison=True,
+                                q_fp8=True), parts)
+
+
 def test_fp8_cache_forced_splits(mla):
     check_full(mla, W.make_case([2000, 33, 700, 4000, 129], h=128, kv="fp8", seed=32, poison=True), 7)
 
@@ -179,6 +196,81 @@ def test_bad_page_id_is_reported_not_faulted(mla):
     assert mla.read_device_error() == 0   # the word clears on read
 
 
+@pytest.mark.parametrize("lens,h,q_len", [([37, 130], 16, 1), ([1, 63, 64, 65, 127, 128, 129], 128, 1),
+                                         ([1000, 62, 129, 1], 128, 4)])
+def test_e5m2_cache(mla, lens, h, q_len):
+    """An e5m2 cache (the other fp8 type the backend accepts) with its per-tensor scale."""
+    check_full(mla, W.make_case(lens, h=h, q_len=q_len, kv="e5m2", verify=q_len > 1, seed=53, poison=True))
+
+
+def test_e5m2_cache_forced_splits(mla):
+    check_full(mla, W.make_case([2000, 33, 700, 4000, 129], h=128, kv="e5m2", seed=54, poison=True), 7)
+
+
+# ------------------------------------------------------------------ KV-cache write
+def _raw(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.uint8)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float8_e4m3fn, torch.float8_e5m2])
+@pytest.mark.parametrize("loc_dtype", [torch.int32, torch.int64])
+def test_set_kv_buffer_bit_exact(mla, dtype, loc_dtype):
+    """set_kv_buffer writes exactly the oracle's rows (fp8: k / k_scale rounded in float32 to
+    the nearest code, ties to even, saturating) and nothing else."""
+    rng = np.random.default_rng(60)
+    slots, n = 64 * 40, 37
+    pool = torch.from_numpy(rng.standard_normal((slots, 576)).astype(np.float32)).to(dtype)
+    loc = torch.from_numpy(rng.choice(slots, size=n, replace=False)).to(loc_dtype)
+    k = torch.from_numpy((rng.standard_normal((n, 576)) * 3).astype(np.float32)).to(torch.bfloat16)
+    k[0, :8] = torch.tensor([1e30, -1e30, 0.0, -0.0, 1e-30, 448.0, 449.0, 57344.0]).to(torch.bfloat16)
+    scale = torch.tensor([0.0123], dtype=torch.float32) if dtype != torch.bfloat16 else None
+    ref = oracle.set_kv_buffer(pool.clone(), loc, k, float(scale[0]) if scale is not None else None)
+    got = mla.set_kv_buffer(pool.cuda(), loc.cuda(), k.cuda(), scale.cuda() if scale is not None else None)
+    torch.cuda.synchronize()
+    assert torch.equal(_raw(got.cpu()), _raw(ref))
+    assert mla.read_device_error() == 0
+
+
+def test_set_kv_buffer_out_of_range_slot_is_reported(mla):
+    pool = torch.zeros((128, 576), dtype=torch.bfloat16, device="cuda")
+    k = torch.ones((3, 576), dtype=torch.bfloat16, device="cuda")
+    loc = torch.tensor([5, 128, -1], dtype=torch.int64, device="cuda")
+    mla.set_kv_buffer(pool, loc, k)
+    torch.cuda.synchronize()
+    assert mla.read_device_error() == 256
+    assert torch.all(pool[5] == 1) and int(torch.count_nonzero(pool)) == 576
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "e5m2"])
+def test_kv_write_then_attention(mla, kv):
+    """One decode step as the backend runs it: each request's newest token (position L - 1) is
+    written into the pool by set_kv_buffer, then attention reads it as the last key; the
+    oracle does the same on its own copy of the pool."""
+    wl = W.make_case([500, 64, 1300, 2], h=128, kv=kv, seed=61)
+    rng = np.random.default_rng(61)
+    k_new = torch.from_numpy(rng.standard_normal((wl.bs, 576)).astype(np.float32)).to(torch.bfloat16)
+    slots = torch.tensor([int(wl.req_to_token[wl.req_pool_indices[b], int(wl.cache_seqlens[b]) - 1])
+                          for b in range(wl.bs)], dtype=torch.int64)
+    scale = wl.descale_k
+    ref_pool = oracle.set_kv_buffer(wl.kv_cache.clone().reshape(-1, 576), slots, k_new,
+                                    float(scale[0]) if scale is not None else None)
+    g = wl.to("cuda")
+    mla.set_kv_buffer(g.kv_cache.reshape(-1, 576), slots.cuda(), k_new.cuda(), g.descale_k)
+    wl.kv_cache = ref_pool.reshape(wl.kv_cache.shape)
+    bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages)
+    md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, 1, wl.is_fp8)
+    o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                                  True, g.descale_q, g.descale_k)
+    torch.cuda.synchronize()
+    assert torch.equal(_raw(g.kv_cache.cpu()), _raw(wl.kv_cache))
+    ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
+                                       wl.cache_seqlens, wl.softmax_scale, True, kv_is_fp8=wl.is_fp8,
+                                       descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
+                                       descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, f"write then attend ({kv})")
+    assert mla.read_device_error() == 0
+
+
 # ------------------------------------------------------------------ full-size workloads
 def sample_rows(wl, n, seed):
     """n random rows, plus, for every request and every query position, its first head, its
@@ -206,6 +298,18 @@ def test_full_size_workload_sampled(mla, index):
     assert_close(o_rows, lse_rows, ref_o, ref_lse, wl.name)
     # properties that hold at any size: finite outputs everywhere, lse at least the
     # log of one allowed key's weight (lse > -inf) for every live row
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    assert mla.read_device_error() == 0
+
+
+def test_full_size_fp8_queries_sampled(mla):
+    """The fp8-cache workload with its queries handed over as e4m3 codes."""
+    wl = W.make_workload(4, q_fp8=True)
+    bt, md, ns, o, lse = run_path(mla, wl)
+    check_metadata(mla, wl, bt, md, ns)
+    rows = sample_rows(wl, 96, seed=44)
+    ref_o, ref_lse = oracle_rows(wl, rows)
+    assert_close(o.reshape(-1, 512)[rows], lse.reshape(-1)[rows], ref_o, ref_lse, wl.name)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     assert mla.read_device_error() == 0
 
@@ -322,6 +426,65 @@ def test_planner_random_batches(mla):
         assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits differs (bs {bs}, parts {parts})"
 
 
+# ------------------------------------------------------------------ one-launch metadata
+@pytest.mark.parametrize("index", [1, 2, 3, 4, 5])
+def test_one_launch_metadata_matches_oracle(mla, index):
+    """build_decode_metadata: page table, int32 lengths and plan in one launch, bit-exact."""
+    wl = W.make_workload(index)
+    g = wl.to("cuda")
+    bt, cl, md, ns = mla.build_decode_metadata(g.req_to_token, g.req_pool_indices, g.seq_lens,
+                                               wl.max_pages, wl.q_len * wl.h, 1, wl.is_fp8,
+                                               seq_len_add=wl.num_draft_tokens)
+    torch.cuda.synchronize()
+    check_metadata(mla, wl, bt.cpu().numpy(), md.cpu().numpy(), ns.cpu().numpy())
+    assert np.array_equal(cl.cpu().numpy(), wl.cache_seqlens.numpy())
+    assert mla.read_device_error() == 0
+
+
+def _random_tables(rng, lens, extra_rows=3):
+    """req_to_token / req_pool_indices for the given lengths: whole pages drawn from a
+    shuffled pool, slots in order inside a page (no KV values: metadata only)."""
+    pages = [-(-int(L) // 64) for L in lens]
+    perm = rng.permutation(max(1, int(sum(pages) * 1.25) + 1))
+    rows = len(lens) + extra_rows
+    width = max(1, max(pages, default=1)) * 64
+    r2t = np.zeros((rows, width), dtype=np.int32)
+    rpi = rng.permutation(rows)[:len(lens)].astype(np.int64)
+    cur = 0
+    for b, n in enumerate(pages):
+        pg = perm[cur:cur + n]
+        cur += n
+        if n:
+            r2t[rpi[b], :64 * n] = (pg[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+    return torch.from_numpy(r2t), torch.from_numpy(rpi)
+
+
+def test_one_launch_metadata_random_batches(mla):
+    """The one-launch metadata against the oracle on random batches: zero, one-block and long
+    requests, 1 to 2500 requests (both planner walks), 1 to 148 parts, a draft-token offset."""
+    rng = np.random.default_rng(20261203)
+    for t in range(60):
+        bs = int(rng.integers(1, 2500 if t % 10 == 0 else 200))
+        kind = rng.integers(0, 3, size=bs)
+        lens = np.where(kind == 0, 0, np.where(kind == 1, rng.integers(1, 65, size=bs),
+                                                rng.integers(1, 8193, size=bs)))
+        add = int(rng.integers(0, 5)) if t % 3 == 0 else 0
+        parts = int(rng.integers(1, 149))
+        r2t, rpi = _random_tables(rng, lens + add)
+        sl = torch.tensor(lens, dtype=torch.int32)
+        max_pages = max(1, -(-int((lens + add).max()) // 64))
+        bt, cl, md, ns = mla.build_decode_metadata(r2t.cuda(), rpi.cuda(), sl.cuda(), max_pages, 128,
+                                                   seq_len_add=add, num_parts=parts)
+        torch.cuda.synchronize()
+        ref_bt = oracle.build_block_table(r2t, rpi, sl, max_pages, seq_len_add=add)
+        ref_md, ref_ns = oracle.get_mla_metadata(lens + add, parts)
+        assert np.array_equal(bt.cpu().numpy(), ref_bt), f"batch {t}: page table"
+        assert np.array_equal(cl.cpu().numpy(), lens + add), f"batch {t}: lengths"
+        assert np.array_equal(md.cpu().numpy(), ref_md), f"batch {t}: plan (bs {bs}, parts {parts})"
+        assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits"
+    assert mla.read_device_error() == 0
+
+
 # ------------------------------------------------------------------ repeated calls, one workspace
 def test_repeated_calls_on_one_workspace_are_identical(mla):
     """The path has no atomics and a fixed split order, so repeated calls must agree bit for
@@ -332,11 +495,12 @@ def test_repeated_calls_on_one_workspace_are_identical(mla):
     bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages)
     parts = 9   # forces several pieces per request
     md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, num_parts=parts)
-    ws = torch.empty((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), dtype=torch.uint8, device="cuda")
+    arrival = -(-wl.bs * 1 * 2 * 4 // 256) * 256   # leading arrival words [bs, query tiles, 2]
     outs = []
     for k in range(3):
         if k == 2:
-            ws.fill_(0xFF)   # a workspace full of NaN patterns must not matter either
+            ws[arrival:].fill_(0xFF)   # partials full of NaN patterns must not matter either
         o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
                                       wl.causal, workspace=ws)
         torch.cuda.synchronize()
@@ -344,4 +508,29 @@ def test_repeated_calls_on_one_workspace_are_identical(mla):
     for o, lse in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1]), "repeated calls differ"
     assert int(ns[-1]) > wl.bs, "the case should split requests"
+    assert torch.count_nonzero(ws[:arrival]) == 0, "every call leaves the arrival words zero"
     assert mla.read_device_error() == 0
+
+
+def test_unzeroed_workspace_is_reported(mla):
+    """A workspace whose arrival words are not zero (never zero-filled) is reported in the
+    error word; zero-filling it makes the next call correct again."""
+    wl = W.make_case([700, 1500, 64, 2300, 1], 128, seed=78)
+    g = wl.to("cuda")
+    bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages)
+    parts = 9
+    md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, num_parts=parts)
+    ws = torch.full((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                         wl.causal, workspace=ws)
+    torch.cuda.synchronize()
+    assert mla.read_device_error() & 128
+    ws.zero_()
+    o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                                  wl.causal, workspace=ws)
+    torch.cuda.synchronize()
+    assert mla.read_device_error() == 0
+    ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
+                                       wl.cache_seqlens, wl.softmax_scale, wl.causal)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "after zero-fill")

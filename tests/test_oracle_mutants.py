@@ -30,8 +30,13 @@ MUTANTS = {
                               "double w = exp(lse_parts[k] - m);"),
     "fp8_query_neighbours_swapped": ("qd[d] = q_is_fp8 ? e4m3_bits_to_double(((const uint8_t*)q_row)[d])",
                                      "qd[d] = q_is_fp8 ? e4m3_bits_to_double(((const uint8_t*)q_row)[d ^ 1])"),
-    "descale_k_dropped": ("? e4m3_bits_to_double(kv[slot * dq + d]) * descale_k\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc",
-                          "? e4m3_bits_to_double(kv[slot * dq + d])\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc"),
+    "descale_k_dropped": ("? fp8_bits_to_double(kv[slot * dq + d], kv_format) * descale_k\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc",
+                          "? fp8_bits_to_double(kv[slot * dq + d], kv_format)\n                                  : bf16_bits_to_double(((const uint16_t*)kv)[slot * dq + d]);\n            acc"),
+    "e5m2_exponent_bias": ("v = ldexp((double)(4 + m), e - 17);", "v = ldexp((double)(4 + m), e - 16);"),
+    "quantize_ties_away_from_zero": ("if (err < best_err || (err == best_err && (code & 1) == 0)) {",
+                                     "if (err < best_err || (err == best_err && code > best)) {"),
+    "set_kv_slot_ignored": ("int64_t slot = cache_loc[i];", "int64_t slot = i;"),
+    "set_kv_scale_multiplied": ("if (has_scale) x = x / k_scale;", "if (has_scale) x = x * k_scale;"),
 }
 
 

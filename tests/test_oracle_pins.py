@@ -36,6 +36,65 @@ def test_bf16_decoding_matches_torch():
     assert np.array_equal(ref[~nan], got[~nan])
 
 
+def test_e5m2_decoding_matches_torch_for_all_codes():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e5m2).to(torch.float64).numpy()
+    got = np.array([oracle.e5m2_to_double(int(c)) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])   # infinities included
+
+
+@pytest.mark.parametrize("fmt,tdt,top", [("e4m3", torch.float8_e4m3fn, 448.0),
+                                          ("e5m2", torch.float8_e5m2, 57344.0)])
+def test_fp8_rounding_matches_torch_and_saturates(fmt, tdt, top):
+    """Round-to-nearest-even of in-range values agrees with torch's cast; exact midpoints
+    between neighbouring codes go to the even code; beyond the range it saturates."""
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(3000) * top / 8, rng.standard_normal(3000) * 1e-3,
+                        [0.0, -0.0, top, -top, 1e-12, -1e-12]])
+    x = x[np.abs(x) <= top]
+    ref = torch.from_numpy(x.astype(np.float32)).to(tdt).view(torch.uint8).numpy()
+    got = np.array([oracle.quantize_fp8(float(np.float32(v)), fmt) for v in x], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+    # midpoints: between every pair of neighbouring positive finite codes
+    dec = oracle.e4m3_to_double if fmt == "e4m3" else oracle.e5m2_to_double
+    vals = [dec(c) for c in range(0x80)]
+    finite = [c for c in range(0x80) if math.isfinite(vals[c])]
+    for a, b in zip(finite[:-1], finite[1:]):
+        mid = (vals[a] + vals[b]) / 2
+        want = a if a % 2 == 0 else b
+        assert oracle.quantize_fp8(mid, fmt) == want, (fmt, a, b)
+        assert oracle.quantize_fp8(-mid, fmt) == want | 0x80
+    assert oracle.quantize_fp8(1e30, fmt) == finite[-1]
+    assert oracle.quantize_fp8(-1e30, fmt) == finite[-1] | 0x80
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float8_e4m3fn, torch.float8_e5m2])
+def test_set_kv_buffer_writes_the_new_rows(dtype):
+    """Rows cache_loc[i] receive token i's row (k / k_scale rounded to an fp8 pool's format, as
+    torch's cast rounds it); every other row, and out-of-range slots, are left alone."""
+    rng = np.random.default_rng(11)
+    slots, dim, n = 50, 576, 7
+    pool = torch.from_numpy(rng.standard_normal((slots, dim)).astype(np.float32)).to(dtype)
+    before = pool.clone()
+    loc = np.array([3, 17, 0, 49, 8, 60, -2], dtype=np.int64)   # the last two are outside the pool
+    k = torch.from_numpy(rng.standard_normal((n, dim)).astype(np.float32)).to(torch.bfloat16)
+    scale = 0.0125 if dtype != torch.bfloat16 else None
+    oracle.set_kv_buffer(pool, loc, k, scale)
+    for i, s in enumerate(loc):
+        if not 0 <= s < slots:
+            continue
+        if dtype == torch.bfloat16:
+            want = k[i]
+        else:
+            want = (k[i].float() / torch.tensor(scale, dtype=torch.float32)).to(dtype)
+        assert torch.equal(pool[s].view(torch.uint8 if dtype != torch.bfloat16 else torch.int16),
+                           want.view(torch.uint8 if dtype != torch.bfloat16 else torch.int16)), (i, s)
+    untouched = [s for s in range(slots) if s not in set(int(v) for v in loc)]
+    assert torch.equal(pool[untouched].float(), before[untouched].float())
+
+
 # ---------------------------------------------------------------- page table
 def _parse_page_table_golden():
     lines = [l.split("#")[0].strip() for l in open(os.path.join(GOLDEN, "page_table_small.txt"))]
@@ -386,6 +445,22 @@ def test_fp8_equals_bf16_on_dequantized_cache():
     b16.kv_cache, b16.descale_k, b16.descale_q = deq, None, None
     ob, lb = run_oracle(b16)
     assert np.array_equal(o8, ob) and np.array_equal(l8, lb)
+
+
+def test_e5m2_cache_equals_bf16_on_dequantized_cache():
+    """An e5m2 cache (the other fp8 format the backend accepts) with its descale equals the
+    bf16 oracle on a cache holding the dequantised values (e5m2 x scale is exact in bf16
+    for a power-of-two scale)."""
+    wl = W.make_case([100, 37], h=8, seed=12)
+    codes = (wl.kv_cache.float() * 4).to(torch.float8_e5m2)
+    scale = 0.25
+    deq = (codes.float() * scale).to(torch.bfloat16)
+    assert torch.equal(deq.float(), codes.float() * scale)
+    o8, l8 = oracle.mla_decode(wl.q, codes, wl.req_to_token, wl.req_pool_indices, wl.cache_seqlens,
+                               wl.softmax_scale, True, kv_is_fp8=True, descale_k=scale)
+    ob, lb = oracle.mla_decode(wl.q, deq, wl.req_to_token, wl.req_pool_indices, wl.cache_seqlens,
+                               wl.softmax_scale, True)
+    assert np.allclose(o8, ob, rtol=0, atol=1e-12) and np.allclose(l8, lb, rtol=0, atol=1e-12)
 
 
 def test_fp8_query_equals_bf16_query_on_its_values():
