@@ -291,6 +291,20 @@ MLA_API mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t
                                        mla_stream_t stream);
 
 /*
+ * Test hooks for the failure path of mla_decode_paged; not for production use.  They set
+ * process-wide values that every later mla_decode_paged launch (from any thread) takes:
+ *   wait_budget_ns  the budget of one pipeline wait (0 restores the default of 2 s);
+ *   withhold_tile   the index (within a scheduler part, counting from 0) of a tile whose page
+ *                   load the leader CTA of every pair does not issue, so that the wait for it
+ *                   runs out (-1 restores normal operation).
+ * When a wait runs out the CTA records MLA_DEVERR_WAIT_TIMEOUT, both CTAs of the pair stop at
+ * their next wait, let their issued copies land, release their tensor memory and return; the
+ * call's outputs are then undefined and its workspace must be zero-filled again.  Host-only,
+ * no synchronisation.  Returns MLA_ERR_INVALID_ARG for withhold_tile < -1.
+ */
+MLA_API mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile);
+
+/*
  * Read and clear the sticky device error word of the current device (a bitwise OR of
  * MLA_DEVERR_* since the last read).  Synchronises `stream`, so it is not for use inside
  * graph capture.  *code_out (host) receives the word; returns MLA_ERR_DEVICE_CHECK when it

@@ -83,6 +83,8 @@ def library() -> ctypes.CDLL:
     lib.mla_decode_paged.restype = I32
     lib.mla_set_kv_buffer.argtypes = [P, I32, I64, P, I32, I32, P, I64, P, P]
     lib.mla_set_kv_buffer.restype = I32
+    lib.mla_set_test_hooks.argtypes = [ctypes.c_uint64, I32]
+    lib.mla_set_test_hooks.restype = I32
     lib.mla_read_device_error.argtypes = [ctypes.POINTER(I32), P]
     lib.mla_read_device_error.restype = I32
     _lib = lib
@@ -317,6 +319,12 @@ def set_kv_buffer(k_cache: torch.Tensor, cache_loc: torch.Tensor, k: torch.Tenso
                                        _ptr(loc), _index_dtype(loc), n, _ptr(k), k.stride(0), _ptr(k_scale),
                                        _stream(k_cache.device)), "mla_set_kv_buffer")
     return k_cache
+
+
+def set_test_hooks(wait_budget_ns: int = 0, withhold_tile: int = -1) -> None:
+    """Test-only: the pipeline wait budget (0: the default 2 s) and a tile whose page load the
+    leader CTAs withhold (-1: none) for every later attention launch in this process."""
+    _check(library().mla_set_test_hooks(int(wait_budget_ns), int(withhold_tile)), "mla_set_test_hooks")
 
 
 def read_device_error(device=None) -> int:

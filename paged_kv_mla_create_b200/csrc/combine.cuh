@@ -194,6 +194,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                       const int32_t* __restrict__ num_splits, int32_t rows,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+    // launched as a programmatic dependent of the attention kernel: wait for all of it
+    pdl_wait_prerequisites();
     const uint64_t read_pol = l2_policy_evict_first();   // the partials are read once
     const int b = blockIdx.y;
     const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);

@@ -113,14 +113,20 @@ enum : int {
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
     kBarPartial,                        // local: the 128 softmax threads stored a split piece
     kBarVWiden,                         // local, e4m3 q: warps 8..11 read their raw V chunks
+    kBarFold,                           // local: the other piece's partial rows landed (fold-in merge)
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
 };
 
-// After the barriers: tensor-memory base, abort flag, pending-merge count, and up to two
-// pending merges (request, first split slot, pieces): only a part's first and last units
-// can be pieces of split requests.
+// After the barriers: tensor-memory base, abort flag, pending-merge count, up to two pending
+// merges (request, first split slot, pieces): only a part's first and last units can be pieces
+// of split requests, and the fold decision of the current epilogue.
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kMiscFold = 8;          // int index into the misc area: the fold-in decision
+// Fold-in merge: the other piece's partial rows, copied into the idle K ring one 2 KB row per
+// copy at this stride (16 bytes of padding rotate the rows' banks).
+constexpr int kFoldRowStride = kDv * 4 + 16;
+static_assert(kCtaRows * kFoldRowStride <= kKSlots * kKSlotBytes, "fold-in rows fit the K ring");
 constexpr int kMaxPendingMerges = 2;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -218,6 +224,8 @@ struct Params {
     float* part_o;                 // [splits, rows, 512]
     float* part_lse;               // [splits, rows]
     int32_t* arrivals;             // [bs, query tiles, 2]: split pieces arrived (zero between calls)
+    uint64_t wait_budget_ns;       // budget of one pipeline wait
+    int32_t withhold_tile;         // test hook: the leader's K load of this tile is not issued (-1: none)
 };
 
 // The work units of a part, identical in every role: request b, block range [kb0, kb1).
@@ -323,6 +331,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const bool leader = rank == 0;
     const int part = blockIdx.x >> 1;
     const int mtile = blockIdx.y;
+    // The merge kernel that follows waits for this whole grid anyway; let it be scheduled
+    // now, so that its launch overlaps this kernel.
+    pdl_launch_dependents();
+    // The part's plan row first, and the first request's length and page ids it points at
+    // fetched into L2, so that their latency overlaps the set-up below rather than delaying the
+    // first page load.
+    bool md_ok = true;
+    UnitIter iter = make_iter(p, part, md_ok);
+    if (warp == 0 && md_ok && iter.b < p.bs) {
+        if (lane == 0) prefetch_l2(p.cache_seqlens + iter.b);
+        const int blk = iter.k0 + lane;
+        if (blk < p.max_pages) prefetch_l2(p.block_table + (int64_t)iter.b * p.bt_stride + blk);
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
@@ -338,6 +359,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // bf16: the Q TMA + 4 warps' tensor-memory stores; e4m3 cache: the 4 warps; e4m3 q: the TMA
         mbar_init(bar(kBarQFull), kFp8Q ? 1 : (kFp8 ? 0 : 1) + 4);
         mbar_init(bar(kBarVWiden), 128);
+        mbar_init(bar(kBarFold), 1);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
@@ -369,9 +391,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // (the partner's flag was zeroed before the cluster barrier above)
+    const AbortCtl actl{abort_flag, map_to_cta(smem_u32(tmem_slot + 1), rank ^ 1u), p.wait_budget_ns};
 
-    bool md_ok = true;
-    UnitIter iter = make_iter(p, part, md_ok);
     const uint64_t kv_pol = l2_policy_evict_first();
     const uint64_t part_pol = l2_policy_evict_last();
     if (!md_ok && threadIdx.x == 0) raise_error(8 /* MLA_DEVERR_BAD_METADATA */);
@@ -413,9 +435,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 int ok = 1;
                 const int s = (int)(g & 1u);
                 const uint32_t slot = sbase + kOffK + s * kKSlotBytes;
+                // test hook: the leader withholds one tile's page, so a wait runs out
+                const bool withhold = leader && (int)g == p.withhold_tile;
                 if (lane == 0) {
-                    ok = mbar_wait_bounded(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, abort_flag);
-                    if (ok) {
+                    ok = mbar_wait_bounded(bar(kBarKEmpty + s), ((g >> 1) & 1u) ^ 1u, actl);
+                    if (ok && !withhold) {
                         if constexpr (kFp8 && !kFp8Q) {
                             mbar_arrive_expect_tx(bar(kBarKRaw + s), kPage8Bytes);
                             tma_load_3d_hint(slot + kRaw8Off, &k_map, bar(kBarKRaw + s), 0, row, 0, kv_pol);
@@ -435,7 +459,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 if constexpr (kFp8 && !kFp8Q) {
                     // the whole warp widens the page in place, then signals the leader
-                    const bool landed = mbar_wait_bounded(bar(kBarKRaw + s), (g >> 1) & 1u, abort_flag);
+                    const bool landed = mbar_wait_bounded(bar(kBarKRaw + s), (g >> 1) & 1u, actl);
                     if (!__all_sync(0xffffffffu, landed)) {
                         alive = false;
                         break;
@@ -494,7 +518,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             const int n = tiles_of(kb0, kb1);
             if (n <= 0) continue;
             // ---- Q of the unit
-            if (uq > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (uq - 1) & 1u, abort_flag)) break;
+            if (uq > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (uq - 1) & 1u, actl)) break;
             tc_fence_after();
             if constexpr (kFp8Q) {
                 // e4m3 codes of the CTA's 64 rows, all 576 columns: one 36 KB TMA (64-byte swizzle)
@@ -568,7 +592,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     if (quarter == 3) {
                         int ok = 1;
                         if (lane == 0) {
-                            ok = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                            ok = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, actl);
                             if (ok) {
                                 if (leader) mbar_arrive_expect_tx(bar(kBarVFull + s), 2 * 2 * 2 * kBox);
                                 const int32_t row = pg >= 0 ? pg * kPage : (int32_t)(p.num_pages * kPage);
@@ -596,7 +620,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                              p.kv + ((int64_t)pg * kPage + row) * kDqk + chunk * 64 + q4 * 16))
                                        : make_uint4(0, 0, 0, 0);
                     }
-                    const bool done = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, abort_flag);
+                    const bool done = mbar_wait_bounded(bar(kBarQKDone + s), (g >> 1) & 1u, actl);
                     if (!__all_sync(0xffffffffu, done)) {
                         alive = false;
                         break;
@@ -611,7 +635,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         uint4 w[8];
                         load_chunk_sw64(slot + kRaw8Off + oc * kChunk8, lane, w);
                         mbar_arrive(bar(kBarVWiden));
-                        const bool read_all = mbar_wait_bounded(bar(kBarVWiden), g & 1u, abort_flag);
+                        const bool read_all = mbar_wait_bounded(bar(kBarVWiden), g & 1u, actl);
                         if (!__all_sync(0xffffffffu, read_all)) {
                             alive = false;
                             break;
@@ -761,9 +785,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     t_idle = global_timer_ns();
                 } else {
                     if (*abort_flag) break;
-                    if (global_timer_ns() - t_idle > kWaitBudgetNs) {
-                        raise_error(16 /* MLA_DEVERR_WAIT_TIMEOUT */);
-                        *abort_flag = 1;
+                    if (global_timer_ns() - t_idle > actl.budget_ns) {
+                        raise_abort(actl);
                         break;
                     }
                 }
@@ -806,13 +829,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 continue;
             }
             const int L = p.cache_seqlens[ub];
+            // where the unit's result goes, read now so that the epilogue does not wait for it
+            bool last_unit;
+            {
+                UnitIter rest = iter;
+                int b_, a_, c_;
+                last_unit = !rest.next(b_, a_, c_);
+            }
+            const int pieces = p.num_splits[ub + 1] - p.num_splits[ub];
+            const bool direct = pieces == 1;
+            const int split = p.num_splits[ub] + (ub == iter.first_b ? p.md[8 * part + 4] : 0);
             int lim = p.causal ? L - p.q_len + iq + 1 : L;
             if (lim > L) lim = L;
             if (lim > kb1 * kPage) lim = kb1 * kPage;   // keys of this unit only
             float m_run = -INFINITY, l_half = 0.f;
             for (int i = 0; i < n; ++i, ++g) {
                 const uint32_t sb = g & 1u;
-                if (!mbar_wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, abort_flag)) {
+                if (!mbar_wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, actl)) {
                     alive = false;
                     break;
                 }
@@ -844,7 +877,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 // partner thread t ^ 64 holds the other 64 tokens of this row
                 xmax[sb * 128 + t] = hmax;
                 mbar_arrive(bar(kBarXchg + sb));
-                if (!mbar_wait_bounded(bar(kBarXchg + sb), (g >> 1) & 1u, abort_flag)) {
+                if (!mbar_wait_bounded(bar(kBarXchg + sb), (g >> 1) & 1u, actl)) {
                     alive = false;
                     break;
                 }
@@ -871,7 +904,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 l_half += psum;
                 // the P buffer is free, and O holds every PV up to tile g - 1, once PV(g - 1)
                 // has finished
-                if (g >= 1 && !mbar_wait_bounded(bar(kBarPvDone), (g - 1) & 1u, abort_flag)) {
+                if (g >= 1 && !mbar_wait_bounded(bar(kBarPvDone), (g - 1) & 1u, actl)) {
                     alive = false;
                     break;
                 }
@@ -912,96 +945,148 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             }
             if (!alive) break;
             // epilogue of the unit
-            if (!mbar_wait_bounded(bar(kBarOFull), uq & 1u, abort_flag)) break;
+            if (!mbar_wait_bounded(bar(kBarOFull), uq & 1u, actl)) break;
             tc_fence_after();
+            // Fold-in merge: a piece of a two-piece request, in its part's last unit (the K ring
+            // is idle), whose other piece has already stored its partial rows, merges them into
+            // its own O and writes the final o; it stores no partial of its own.
+            int32_t* const arrival = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
+            if (t == 0)
+                pending[kMiscFold] = (!direct && pieces == 2 && pieces <= kFusedMergeMaxPieces && last_unit &&
+                                     ld_acquire_gpu(arrival) == 1) ? 1 : 0;
             xmax[256 + t] = l_half;
             mbar_arrive(bar(kBarLx));
-            if (!mbar_wait_bounded(bar(kBarLx), uq & 1u, abort_flag)) break;
+            if (!mbar_wait_bounded(bar(kBarLx), uq & 1u, actl)) break;
+            const bool fold = pending[kMiscFold] != 0;
             const float l_run = l_half + xmax[256 + (t ^ 64)];
-            const int pieces = p.num_splits[ub + 1] - p.num_splits[ub];
-            const bool direct = pieces == 1;
-            const int split = p.num_splits[ub] + (ub == iter.first_b ? p.md[8 * part + 4] : 0);
-            const float inv = l_run > 0.f ? dk / l_run : 0.f;
-            const float lse_val = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f
-                                              : -INFINITY;
-            // Each warp holds 32 rows; a step moves 128 bytes of each row (32 fp32 partial
-            // columns, or 64 bf16 output columns) from tensor memory through a per-warp staging
-            // area, so that every global store writes whole 128-byte lines (8 lanes per row).
+            float inv = l_run > 0.f ? dk / l_run : 0.f;
+            float lse_val = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+            float other_w = 0.f;
+            if (fold) {
+                const int s0 = p.num_splits[ub];
+                const int other = s0 + 1 - (split - s0);
+                const int row_base = mtile * kRows + kCtaRows * (int)rank;
+                const int nrows = min(kCtaRows, p.rows - row_base);
+                if (warp == kSoftmaxWarp0) {
+                    if (lane == 0) mbar_arrive_expect_tx(bar(kBarFold), (uint32_t)nrows * (kDv * 4));
+                    fence_proxy_async_global();   // the acquired partial rows, read by the async proxy
+                    __syncwarp();
+                    for (int r = lane; r < nrows; r += 32)
+                        bulk_load(sbase + kOffK + (uint32_t)(r * kFoldRowStride),
+                                  p.part_o + ((int64_t)other * p.rows + row_base + r) * kDv, kDv * 4, bar(kBarFold));
+                }
+                // merged lse and the two weights (log2 units): own (m_run, l_run), other lse_o
+                const float lse_o = row_valid ? __ldcg(p.part_lse + (int64_t)other * p.rows + rowg) : -INFINITY;
+                const float own2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+                const float oth2 = lse_o * 1.4426950408889634f;
+                const float mx = fmaxf(own2, oth2);
+                if (mx == -INFINITY) {
+                    inv = 0.f;
+                    lse_val = -INFINITY;
+                } else {
+                    const float w_own = fast_exp2(own2 - mx), w_oth = fast_exp2(oth2 - mx);
+                    const float tot = w_own + w_oth;
+                    inv = l_run > 0.f ? dk * w_own / (tot * l_run) : 0.f;
+                    other_w = w_oth / tot;
+                    lse_val = (mx + __log2f(tot)) * 0.69314718055994531f;
+                }
+                if (!mbar_wait_bounded(bar(kBarFold), 0u, actl)) break;   // one fold per CTA at most
+            }
+            const bool write_final = direct || fold;
+            // Each warp holds 32 rows.  A step reads 64 tensor-memory columns of its rows (one
+            // wait) and moves them, 128 bytes of each row at a time (64 bf16 outputs, or 32 fp32
+            // partial columns: two passes), through a per-warp staging area, so that every global
+            // store writes whole 128-byte lines (8 lanes per row).  TMEM columns [128 + 64 st, +64)
+            // hold outputs 256 (st / 2) + 128 half + 64 (st % 2) + [0, 64).
             {
                 const uint32_t stage = sbase + kOffStage + (uint32_t)(warp - kSoftmaxWarp0) * 4096u;
                 const int row0 = mtile * kRows + kCtaRows * (int)rank + 32 * ((warp - kSoftmaxWarp0) & 1);
-                const int steps = direct ? 4 : 8;
 #pragma unroll 1
-                for (int st = 0; st < steps; ++st) {
-                    uint32_t w[32];
-                    int col;
-                    if (direct) {
-                        // 64 columns: TMEM columns [128 + 64 st, +64) = outputs
-                        // 256 (st / 2) + 128 half + 64 (st % 2) + [0, 64)
-                        uint32_t raw[64];
-                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st, *reinterpret_cast<uint32_t(*)[16]>(raw));
-                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(raw + 16));
-                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 32u, *reinterpret_cast<uint32_t(*)[16]>(raw + 32));
-                        tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 48u, *reinterpret_cast<uint32_t(*)[16]>(raw + 48));
-                        tc_wait_ld();
-                        if (st == steps - 1) {
-                            tc_fence_before();
-                            signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));   // O is free for the next unit
-                        }
-#pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv, __uint_as_float(raw[2 * k + 1]) * inv);
-                        col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
-                    } else {
-                        // 32 columns: TMEM columns [128 + 32 st, +32) = outputs
-                        // 256 (st / 4) + 128 half + 32 (st % 4) + [0, 32)
-                        tmem_ld16(tmem + lane_off + kTmemO + 32u * st, *reinterpret_cast<uint32_t(*)[16]>(w));
-                        tmem_ld16(tmem + lane_off + kTmemO + 32u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(w + 16));
-                        tc_wait_ld();
-                        if (st == steps - 1) {
-                            tc_fence_before();
-                            signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));   // O is free for the next unit
-                        }
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * inv);
-                        col = 256 * (st >> 2) + 128 * half + 32 * (st & 3);
+                for (int st = 0; st < 4; ++st) {
+                    uint32_t raw[64];
+                    tmem_ld16(tmem + lane_off + kTmemO + 64u * st, *reinterpret_cast<uint32_t(*)[16]>(raw));
+                    tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(raw + 16));
+                    tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 32u, *reinterpret_cast<uint32_t(*)[16]>(raw + 32));
+                    tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 48u, *reinterpret_cast<uint32_t(*)[16]>(raw + 48));
+                    tc_wait_ld();
+                    if (st == 3) {
+                        tc_fence_before();
+                        signal_leader(kBarOEmpty, 20 + (warp - kSoftmaxWarp0));   // O is free for the next unit
                     }
-                    // this thread's 128 bytes -> staging row `lane` (16-byte unit k at k ^ (lane & 7))
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        st_shared_v4u(stage + (uint32_t)lane * 128u + 16u * ((uint32_t)k ^ ((uint32_t)lane & 7u)),
-                                      w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                    __syncwarp();
-                    // 4 rows per store instruction, 8 lanes (128 contiguous bytes) per row
+                    for (int pass = 0; pass < 2; ++pass) {
+                        if (write_final && pass == 1) break;
+                        uint32_t w[32];
+                        int col;
+                        if (fold) {
+                            // own O (normalised and weighted) + the other piece's row, weighted
+                            col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
+                            const uint32_t orow = sbase + kOffK + (uint32_t)(rloc * kFoldRowStride + col * 4);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int r = 4 * j + (lane >> 3), u = lane & 7;
-                        const int rg = row0 + r;
-                        const uint4 v = ld_shared_v4u(stage + (uint32_t)r * 128u + 16u * ((uint32_t)u ^ ((uint32_t)r & 7u)));
-                        if (rg < p.rows) {
-                            if (direct)
-                                *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
-                            else
-                                st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
+                            for (int k = 0; k < 32; k += 2) {
+                                const uint4 v = ld_shared_v4u(orow + 8u * (uint32_t)k);
+                                w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv + __uint_as_float(v.x) * other_w,
+                                                   __uint_as_float(raw[2 * k + 1]) * inv + __uint_as_float(v.y) * other_w);
+                                w[k + 1] = pack_bf16x2(__uint_as_float(raw[2 * k + 2]) * inv + __uint_as_float(v.z) * other_w,
+                                                       __uint_as_float(raw[2 * k + 3]) * inv + __uint_as_float(v.w) * other_w);
+                            }
+                        } else if (direct) {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv, __uint_as_float(raw[2 * k + 1]) * inv);
+                            col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(raw[32 * pass + k]) * inv);
+                            col = 256 * (st >> 1) + 128 * half + 64 * (st & 1) + 32 * pass;
                         }
+                        // this thread's 128 bytes -> staging row `lane` (16-byte unit k at k ^ (lane & 7))
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            st_shared_v4u(stage + (uint32_t)lane * 128u + 16u * ((uint32_t)k ^ ((uint32_t)lane & 7u)),
+                                          w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        __syncwarp();
+                        // 4 rows per store instruction, 8 lanes (128 contiguous bytes) per row
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int r = 4 * j + (lane >> 3), u = lane & 7;
+                            const int rg = row0 + r;
+                            const uint4 v = ld_shared_v4u(stage + (uint32_t)r * 128u + 16u * ((uint32_t)u ^ ((uint32_t)r & 7u)));
+                            if (rg < p.rows) {
+                                if (write_final)
+                                    *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
+                                else
+                                    st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
+                            }
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
             if (row_valid && half == 0) {
-                if (direct)
+                if (write_final)
                     p.lse[(int64_t)ub * p.rows + rowg] = lse_val;
                 else
                     st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
             }
-            if (!direct && pieces <= kFusedMergeMaxPieces) {
+            if (fold) {
+                // the other piece's partial lines are dead: drop them; the arrival word is reset
+                // for the next call (the other piece counted itself, this one never does)
+                const int row_base = mtile * kRows + kCtaRows * (int)rank;
+                const int nrows = min(kCtaRows, p.rows - row_base);
+                const int s0 = p.num_splits[ub];
+                const int other = s0 + 1 - (split - s0);
+                for (int l = t; l < nrows * 16; l += 128)
+                    discard_l2_line(p.part_o + ((int64_t)other * p.rows + row_base + l / 16) * kDv + (l % 16) * 32);
+                if (t == 0) *arrival = 0;
+            } else if (!direct && pieces <= kFusedMergeMaxPieces) {
                 // This piece's partial rows are written: make them visible device-wide, then
                 // count the arrival.  The CTA whose arrival completes the count merges them.
                 // (An mbarrier, not bar.sync, gathers the 128 threads: a bounded wait can never
                 // strand them if another role gave up.)
                 __threadfence();
                 mbar_arrive(bar(kBarPartial));
-                if (!mbar_wait_bounded(bar(kBarPartial), npartial & 1u, abort_flag)) break;
+                if (!mbar_wait_bounded(bar(kBarPartial), npartial & 1u, actl)) break;
                 ++npartial;
                 if (t == 0) {
                     int32_t* word = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mla_b200.h"
@@ -69,6 +70,10 @@ mla_status_t prepare_decode_kernels() {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Test hooks (mla_set_test_hooks): the wait budget and the withheld tile of later launches.
+std::atomic<uint64_t> g_hook_wait_budget_ns{0};
+std::atomic<int32_t> g_hook_withhold_tile{-1};
 
 // Workspace layout: arrival words int32 [bs, query tiles, 2], then the split partials
 // fp32 [splits, rows, 512] and their lse fp32 [splits, rows], each 256-byte aligned.
@@ -325,6 +330,9 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     p.lse = lse;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.arrivals = reinterpret_cast<int32_t*>(ws);
+    const uint64_t budget = g_hook_wait_budget_ns.load(std::memory_order_relaxed);
+    p.wait_budget_ns = budget ? budget : mla::kWaitBudgetNs;
+    p.withhold_tile = g_hook_withhold_tile.load(std::memory_order_relaxed);
     p.part_o = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q));
     p.part_lse = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q) +
                                           align256(splits * rows * 512 * sizeof(float)));
@@ -343,10 +351,21 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
         mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
-    const dim3 cgrid((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
-    mla::combine_splits_kernel<<<cgrid, mla::kCombineWarps * 32, 0, s>>>(
-        p.part_o, p.part_lse, num_splits, rows, p.out, lse);
-    return from_cuda(cudaGetLastError());
+    // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
+    // the attention kernel runs, it waits on the device for that grid to complete.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
+    cfg.blockDim = dim3(mla::kCombineWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, mla::combine_splits_kernel, (const float*)p.part_o, (const float*)p.part_lse,
+                           num_splits, rows, p.out, lse);
+    return from_cuda(e);
 }
 
 mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slots, const void* cache_loc,
@@ -378,6 +397,13 @@ mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slo
     }
 #undef MLA_KV_LAUNCH
     return from_cuda(cudaGetLastError());
+}
+
+mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile) {
+    if (withhold_tile < -1) return MLA_ERR_INVALID_ARG;
+    g_hook_wait_budget_ns.store(wait_budget_ns, std::memory_order_relaxed);
+    g_hook_withhold_tile.store(withhold_tile, std::memory_order_relaxed);
+    return MLA_OK;
 }
 
 mla_status_t mla_read_device_error(int32_t* code_out, mla_stream_t stream) {

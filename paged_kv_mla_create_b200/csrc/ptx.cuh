@@ -68,25 +68,53 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait budget for one pipeline wait.  Every wait in the kernels is bounded: after this
-// many nanoseconds without the phase completing the waiter records
-// MLA_DEVERR_WAIT_TIMEOUT, raises the CTA's abort flag and returns false; a raised abort
-// flag makes every later wait return false at once so that all roles drain to the exit.
+// Default budget of one pipeline wait.  Every wait in the kernels is bounded: after the budget
+// without the phase completing the waiter records MLA_DEVERR_WAIT_TIMEOUT and raises the abort
+// flag of its CTA and of the pair's other CTA; a raised flag makes every later wait return
+// false at once, so that all roles of both CTAs drain to the exit together.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort_flag) {
+// 4-byte store into shared memory of a CTA of the cluster (cluster address from mapa).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// A CTA's abort state: its own flag, the pair partner's flag (cluster address) and the budget.
+struct AbortCtl {
+    volatile int* flag;
+    uint32_t peer_flag;
+    uint64_t budget_ns;
+};
+
+__device__ __forceinline__ void raise_abort(const AbortCtl& a) {
+    raise_error(16 /* MLA_DEVERR_WAIT_TIMEOUT */);
+    *a.flag = 1;
+    st_cluster_u32(a.peer_flag, 1u);
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, const AbortCtl& a) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (*abort_flag) return false;
+        if (*a.flag) return false;
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitBudgetNs) {
-            raise_error(16 /* MLA_DEVERR_WAIT_TIMEOUT */);
-            *abort_flag = 1;
+        if (global_timer_ns() - t0 > a.budget_ns) {
+            raise_abort(a);
             return false;
         }
     }
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched after this one on the same stream with programmatic stream serialization
+// may be scheduled once every CTA of this grid has issued this (or exited).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grids this one depends on have completed and their memory is visible (a
+// no-op for a kernel launched without programmatic serialization).
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ cluster / DSMEM
@@ -120,10 +148,37 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Ask the L2 to fetch the 128-byte line holding addr (nothing returns to the SM).
+__device__ __forceinline__ void prefetch_l2(const void* addr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (TMA / tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Load with acquire semantics at GPU scope (pairs with a writer's fence before its atomic).
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Order this thread's earlier generic-proxy accesses (here: an acquire of data other CTAs
+// stored) before its later async-proxy (bulk copy) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global memory
+// into this CTA's shared memory, completing on this CTA's mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

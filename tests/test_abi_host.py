@@ -94,6 +94,12 @@ def test_decode_validation_happens_before_any_launch():
     assert _decode(lib, q_len=1, h_q=65535 * 128 + 1) == 2   # more query tiles than grid.y holds
 
 
+def test_test_hooks_validation():
+    lib = mla.library()
+    assert lib.mla_set_test_hooks(0, -2) == 1
+    assert lib.mla_set_test_hooks(0, -1) == 0     # the defaults (no launch involved)
+
+
 def test_set_kv_buffer_validation():
     lib = mla.library()
     kv = lib.mla_set_kv_buffer

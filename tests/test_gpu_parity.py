@@ -391,6 +391,27 @@ def test_misaligned_slots_are_reported(mla):
     assert mla.read_device_error() == 0
 
 
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_wait_that_runs_out_returns_with_an_error(mla, kv):
+    """The failure path without a fault: a test hook makes every pair's leader withhold one
+    page load, so a bounded wait (2 ms here) runs out; both CTAs of each pair stop, the kernel
+    returns, the error word says MLA_DEVERR_WAIT_TIMEOUT, and the next ordinary call (with a
+    zero-filled workspace) is correct again."""
+    wl = W.make_case([2000, 1500, 900], h=128, kv=kv, seed=47)
+    g = wl.to("cuda")
+    bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages)
+    md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, 1, wl.is_fp8, num_parts=2)
+    try:
+        mla.set_test_hooks(2_000_000, 3)
+        mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale, True,
+                             g.descale_q, g.descale_k)
+        torch.cuda.synchronize()
+    finally:
+        mla.set_test_hooks(0, -1)
+    assert mla.read_device_error() & 16
+    check_full(mla, wl, 2)
+
+
 def test_q_out_of_f16_range_is_reported(mla):
     """With an e4m3 cache the product runs in f16: a q value beyond 65504 (made on the host)
     is recorded in the error word instead of silently overflowing."""
