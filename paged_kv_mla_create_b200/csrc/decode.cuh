@@ -325,7 +325,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* pending = reinterpret_cast<int*>(smem + kOffMisc + 8);   // count, then (ub, s0, n) x 2
 
-    const int warp = threadIdx.x >> 5;
+    const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);   // warp-uniform to the compiler
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -674,11 +674,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // S(t) waits for its page, its S buffer (the softmax read S(t - 2)) and, first in a
         // unit, the unit's Q; PV(t) waits for P(t), the partner V of tile t and, first in a
         // unit, the epilogue of the previous unit having read O.
-        if (leader && lane == 0) {
-            // Non-blocking barrier tests at CTA scope: the data behind a barrier the peer
-            // completes is ordered by the peer's fence.proxy.async and the st.async / TMA
-            // complete_tx itself (measured ~1% faster than cluster-scope acquire).
-            auto poll = [](uint32_t b, uint32_t parity) -> bool { return mbar_test_wait(b, parity); };
+        if (leader) {
+            // The whole warp walks the schedule (an elected lane issues each MMA, see
+            // mma_pair_ss).  Non-blocking barrier tests at CTA scope: the data behind a barrier
+            // the peer completes is ordered by the peer's fence.proxy.async and the st.async /
+            // TMA complete_tx itself (measured ~1% faster than cluster-scope acquire); the vote
+            // keeps every decision warp-uniform.
+            auto poll = [](uint32_t b, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_test_wait(b, parity));
+            };
             struct Cursor {
                 UnitIter it;
                 int n, i;
@@ -758,21 +762,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                                                    kIdescQK8, (c | kk) ? 1u : 0u);
                         } else {
 #pragma unroll
-                        for (int c = 0; c < kChunks; ++c) {
-                            if (c < kQLoChunks) {
+                            for (int c = 0; c < kChunks; ++c) {
+                                if (c < kQLoChunks) {
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_pair_ts(d, tmem + kTmemQ + 32u * c + 8u * kk,
-                                                smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
-                                                kFp8 ? kIdescQK16 : kIdescQK, (c | kk) ? 1u : 0u);
-                            } else {
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        mma_pair_ts(d, tmem + kTmemQ + 32u * c + 8u * kk,
+                                                    smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                                    kFp8 ? kIdescQK16 : kIdescQK, (c | kk) ? 1u : 0u);
+                                } else {
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_pair_ss(d, smem_desc_sw128(sbase + kOffQ + (c - kQLoChunks) * kBox + 32u * kk, 16, 1024),
-                                                smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
-                                                kFp8 ? kIdescQK16 : kIdescQK, 1u);
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        mma_pair_ss(d, smem_desc_sw128(sbase + kOffQ + (c - kQLoChunks) * kBox + 32u * kk, 16, 1024),
+                                                    smem_desc_sw128(slot + c * kBox + 32u * kk, 16, 1024),
+                                                    kFp8 ? kIdescQK16 : kIdescQK, 1u);
+                                }
                             }
-                        }
                         }
                         tc_commit_pair(bar(kBarQKDone + s));
                         tc_commit_pair(bar(kBarSFull + sb));
@@ -786,7 +790,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 } else {
                     if (*abort_flag) break;
                     if (global_timer_ns() - t_idle > actl.budget_ns) {
-                        raise_abort(actl);
+                        if (lane == 0) raise_abort(actl);
                         break;
                     }
                 }
@@ -864,15 +868,25 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 tc_fence_before();
                 signal_leader(kBarSFree + sb, 16 + (warp - kSoftmaxWarp0));
-                // scale to log2 units, mask, this half's maximum
+                // scale to log2 units, mask the keys at or past the limit (only a tile that
+                // reaches it has any), this half's maximum
                 const int kbase = (kb0 + 2 * i) * kPage + kPage * half;
-                float hmax = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    float x = s[j] * sl2;
-                    if (kbase + j >= lim) x = -INFINITY;
-                    s[j] = x;
-                    hmax = fmaxf(hmax, x);
+                for (int j = 0; j < 64; j += 2) mul2(s[j], s[j + 1], sl2);
+                if (kbase + 64 > lim) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (kbase + j >= lim) s[j] = -INFINITY;
+                }
+                float hmax;
+                {
+                    float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]);
+#pragma unroll
+                    for (int j = 4; j < 64; j += 4) {
+                        m0 = fmax3(m0, s[j], s[j + 1]);
+                        m1 = fmax3(m1, s[j + 2], s[j + 3]);
+                    }
+                    hmax = fmaxf(m0, m1);
                 }
                 // partner thread t ^ 64 holds the other 64 tokens of this row
                 xmax[sb * 128 + t] = hmax;
@@ -890,18 +904,24 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     l_half *= factor;
                     m_run = m_new;
                 }
-                const bool live = m_run != -INFINITY;
-                float psum = 0.f;
                 // P packed as bf16 pairs into s[0..31] (s[2j], s[2j+1] are read before s[j]
-                // is overwritten, since 2j >= j).
+                // is overwritten, since 2j >= j); nothing but zeros while every key so far is masked.
+                if (m_run != -INFINITY) {
+                    float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float p0 = live ? fast_exp2(s[2 * j] - m_run) : 0.f;
-                    const float p1 = live ? fast_exp2(s[2 * j + 1] - m_run) : 0.f;
-                    psum += p0 + p1;
-                    s[j] = __uint_as_float(kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1));
+                    for (int j = 0; j < 32; ++j) {
+                        float p0 = s[2 * j], p1 = s[2 * j + 1];
+                        sub2(p0, p1, m_run);
+                        p0 = fast_exp2(p0);
+                        p1 = fast_exp2(p1);
+                        add2(ps0, ps1, p0, p1);
+                        s[j] = __uint_as_float(kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1));
+                    }
+                    l_half += ps0 + ps1;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s[j] = 0.f;
                 }
-                l_half += psum;
                 // the P buffer is free, and O holds every PV up to tile g - 1, once PV(g - 1)
                 // has finished
                 if (g >= 1 && !mbar_wait_bounded(bar(kBarPvDone), (g - 1) & 1u, actl)) {
