@@ -114,6 +114,7 @@ enum : int {
     kBarPartial,                        // local: the 128 softmax threads stored a split piece
     kBarVWiden,                         // local, e4m3 q: warps 8..11 read their raw V chunks
     kBarFold,                           // local: the other piece's partial rows landed (fold-in merge)
+    kBarMerge,                          // local: a tail merge's pass of partial rows landed
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
 };
@@ -360,6 +361,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         mbar_init(bar(kBarQFull), kFp8Q ? 1 : (kFp8 ? 0 : 1) + 4);
         mbar_init(bar(kBarVWiden), 128);
         mbar_init(bar(kBarFold), 1);
+        mbar_init(bar(kBarMerge), 1);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
             mbar_init(bar(kBarSFull + j), 1);
@@ -1090,14 +1092,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
             }
             if (fold) {
-                // the other piece's partial lines are dead: drop them; the arrival word is reset
-                // for the next call (the other piece counted itself, this one never does)
-                const int row_base = mtile * kRows + kCtaRows * (int)rank;
-                const int nrows = min(kCtaRows, p.rows - row_base);
-                const int s0 = p.num_splits[ub];
-                const int other = s0 + 1 - (split - s0);
-                for (int l = t; l < nrows * 16; l += 128)
-                    discard_l2_line(p.part_o + ((int64_t)other * p.rows + row_base + l / 16) * kDv + (l % 16) * 32);
+                // the arrival word is reset for the next call (the other piece counted itself,
+                // this one never does)
                 if (t == 0) *arrival = 0;
             } else if (!direct && pieces <= kFusedMergeMaxPieces) {
                 // This piece's partial rows are written: make them visible device-wide, then
@@ -1132,19 +1128,24 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
-    // Merges of the requests whose last piece arrived here, by the whole CTA (the row-max
-    // exchange area is free now and holds the weights).
+    // Merges of the requests whose last piece arrived here, by the whole CTA: the pieces' rows
+    // come in by bulk copies into the now idle Q, K ring and P areas (200 KB, as many rows per
+    // pass as fit); the row-max exchange area holds the weights.
     const int npending = pending[0];
     if (npending > 0 && !*abort_flag) {
         __threadfence();   // the other pieces' partials: their fences preceded their arrivals
         const int row_base = mtile * kRows + kCtaRows * (int)rank;
         const int nrows = min(kCtaRows, p.rows - row_base);
+        uint32_t phase = 0;
+        auto wait = [&](uint32_t b, uint32_t parity) { return mbar_wait_bounded(b, parity, actl); };
         for (int k = 0; k < npending && nrows > 0; ++k) {
             const int mb = pending[1 + 3 * k], s0 = pending[2 + 3 * k], n = pending[3 + 3 * k];
-            merge_rows_cta<kThreads>(p.part_o, p.part_lse, s0, n, p.rows, row_base, nrows,
-                                     p.out + ((int64_t)mb * p.rows + row_base) * kDv,
-                                     p.lse + (int64_t)mb * p.rows + row_base,
-                                     reinterpret_cast<float*>(smem + kOffX), threadIdx.x);
+            if (!merge_rows_cta_bulk<kThreads>(p.part_o, p.part_lse, s0, n, p.rows, row_base, nrows,
+                                               p.out + ((int64_t)mb * p.rows + row_base) * kDv,
+                                               p.lse + (int64_t)mb * p.rows + row_base,
+                                               reinterpret_cast<float*>(smem + kOffX), sbase + kOffQ,
+                                               (uint32_t)(kOffX - kOffQ), bar(kBarMerge), phase, wait, threadIdx.x))
+                break;
         }
     }
     cluster_sync();

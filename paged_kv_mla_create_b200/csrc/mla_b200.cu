@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -354,7 +355,11 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
     // the attention kernel runs, it waits on the device for that grid to complete.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((rows + mla::kCombineWarps - 1) / mla::kCombineWarps, bs);
+    {
+        const int64_t need = ((int64_t)bs * rows + mla::kCombineWarps - 1) / mla::kCombineWarps;
+        // as many CTAs as the attention grid (one per SM)
+        cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)grid.x * grid.y)));
+    }
     cfg.blockDim = dim3(mla::kCombineWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
@@ -364,7 +369,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, mla::combine_splits_kernel, (const float*)p.part_o, (const float*)p.part_lse,
-                           num_splits, rows, p.out, lse);
+                           num_splits, rows, bs, p.out, lse);
     return from_cuda(e);
 }
 

@@ -313,11 +313,6 @@ __device__ __forceinline__ float4 ld_global_nc_v4_hint(const float4* ptr, uint64
     return v;
 }
 
-// Drop a 128-byte L2 line without writing it back (its data is dead).
-__device__ __forceinline__ void discard_l2_line(const void* ptr) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(ptr) : "memory");
-}
-
 // Hint the L2 to fetch a tensor box ahead of its load (no shared memory involved).
 __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t c0, int32_t c1,
                                                 int32_t c2, int32_t c3) {
@@ -435,6 +430,10 @@ __device__ __forceinline__ uint4 ld_shared_v4u(uint32_t addr) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(addr));
     return v;
+}
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+    const uint4 u = ld_shared_v4u(addr);
+    return make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
