@@ -500,6 +500,66 @@ class Case:
         return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
+class _NoGraph:
+    def replay(self):
+        pass
+
+
+class ExtendCase(Case):
+    """Extend with a cached prefix (ragged causal part over the new rows, paged part over the
+    prefix, merge_state): 4 requests of the DeepSeek-V3 decode shape (128 heads, prefixes
+    ~U[1024, 4096]) with 64 new tokens each.  One call is the whole extend (its page tables and
+    plans are built inside it), so the metadata step is empty."""
+
+    def __init__(self, seed, dev, flush_mb):
+        import numpy as np
+        import torch
+        import paged_kv_mla_create_b200 as mla
+        from paged_kv_mla_create_b200 import workloads as W
+        self.mla, self.dev, self.cfg = mla, dev, "extend"
+        rng = np.random.default_rng(seed)
+        prefix = [int(x) for x in rng.integers(1024, 4097, size=4)]
+        e = 64
+        self.host = host = W.make_case(prefix, h=128, q_len=e, verify=True, seed=seed,
+                                       name="extend with cached prefix (bs 4, h 128, prefix ~U[1024, 4096], 64 new tokens, bf16)")
+        self.wl = host.to(dev)
+        pool = host.kv_cache.reshape(-1, 576)
+        slots = torch.tensor([[int(host.req_to_token[host.req_pool_indices[b], prefix[b] + i]) for i in range(e)]
+                              for b in range(host.bs)], dtype=torch.int64)
+        self.k_new = pool[slots.reshape(-1)].reshape(host.bs, e, 576).contiguous().to(dev)
+        self.prefix = torch.tensor(prefix, dtype=torch.int32, device=dev)
+        self.mpp = max(-(-p // 64) for p in prefix)
+        # the prefix rows once, the new rows once, q once; FLOPs of the causal new tokens over both
+        self.kv_bytes, self.q_bytes, self.flops = algorithmic(host)
+        self.o = torch.empty((host.bs, e, host.h, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((host.bs, e, host.h), dtype=torch.float32, device=dev)
+        self.ws = torch.zeros((mla.extend_workspace_bytes(host.bs, e, host.h, self.mpp, mla.sm_count(dev)),),
+                              dtype=torch.uint8, device=dev)
+        self.flush = torch.empty((flush_mb << 20,), dtype=torch.uint8, device=dev)
+        self.flush_rd = torch.ones((flush_mb << 20,), dtype=torch.uint8, device=dev)
+
+    def metadata(self, w):
+        pass
+
+    def attention(self, w, o=None, lse=None):
+        self.mla.extend_paged_prefix(w.q, self.k_new, w.kv_cache, w.req_to_token, w.req_pool_indices, self.prefix,
+                                     self.mpp, self.host.softmax_scale, out=self.o if o is None else o,
+                                     lse=self.lse if lse is None else lse, workspace=self.ws)
+
+    def capture(self):
+        import torch
+        stream = torch.cuda.current_stream(self.dev)
+        cap = torch.cuda.Stream(self.dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            self.attention(self.wl)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize(self.dev)
+        self.g_meta, self.g_attn = _NoGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_attn):
+            self.attention(self.wl)
+
+
 def config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src):
     attn_s = attn_ms * 1e-3
     return {"workload": case.host.name, "us_per_call": attn_ms * 1e3,
@@ -561,6 +621,17 @@ def run_b200(args):
             per_config[f"{cfg}q8" if q8 else str(cfg)] = config_entry(c, sm, am, mm, ck, peaks, peak_src)
             del c
             torch.cuda.empty_cache()
+        # the extend piece (new tokens over their own rows and a cached prefix, merged)
+        c = ExtendCase(replica_seed(2, rank) + 7, dev, args.flush_mb)
+        sm, am, mm, ck = c.time_steps(max(1, min(K, args.per_config_steps)), max(3, min(args.warmup, 5)), world,
+                                      ClockSampler(gpu_id_for(dev)))
+        e = mla.read_device_error(dev)
+        sm, am, mm, e = reduce_max_over_ranks([sm, am, mm, float(e)], dev, world)
+        if e:
+            raise RuntimeError(f"device error word {int(e)} after the extend workload")
+        per_config["extend"] = config_entry(c, sm, am, mm, ck, peaks, peak_src)
+        del c
+        torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:

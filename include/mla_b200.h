@@ -291,6 +291,68 @@ MLA_API mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t
                                        mla_stream_t stream);
 
 /*
+ * merge_state (flashinfer_backend.py, forward_extend: o, _ = merge_state(o1, s1, o2, s2)): the
+ * exact log-sum-exp merge of two partial attention results of the same rows,
+ *     lse = ln(exp(lse_a) + exp(lse_b)),   o = exp(lse_a - lse) o_a + exp(lse_b - lse) o_b.
+ *   o_a, o_b      bf16 [rows, head_dim_v], 16-byte aligned; lse_a, lse_b fp32 [rows], natural
+ *                 log, -inf for a part that saw no key
+ *   head_dim_v    512 (else MLA_ERR_UNSUPPORTED)
+ *   o, lse        bf16 [rows, head_dim_v] (16-byte aligned) and fp32 [rows], written; a row with
+ *                 no key in either part gets o = 0 and lse = -inf.
+ * The weights are computed in fp32 from the max-shifted lse values; one warp per row.
+ */
+MLA_API mla_status_t mla_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                                     int64_t rows, int32_t head_dim_v, void* o, float* lse, mla_stream_t stream);
+
+/*
+ * Bytes of workspace mla_extend_paged_prefix needs (256-byte aligned parts: a padded copy of the
+ * new rows when e is not a multiple of 64, the page tables, lengths and plans of both parts,
+ * two mla_decode_paged workspaces and the two partial results).  Pure host function; returns 0
+ * on a non-positive bs, e, h_q or sm_count or a negative max_prefix_pages.
+ */
+MLA_API size_t mla_extend_workspace_bytes(int32_t bs, int32_t e, int32_t h_q, int32_t max_prefix_pages,
+                                          int32_t sm_count);
+
+/*
+ * Extend with a cached prefix (flashinfer_backend.py, forward_extend, the ragged-plus-paged
+ * branch), in MLA form: each request has prefix_lens[b] latent rows already in the paged pool
+ * and e new tokens; the new tokens' queries attend
+ *   (1) the new tokens' own latent rows k_new, causally (new token i sees new tokens 0 .. i):
+ *       the ragged part, o1 / s1;
+ *   (2) the whole cached prefix, non-causally: the paged part, o2 / s2;
+ * and the result is merge_state(o1, s1, o2, s2) -- exactly attention over the prefix followed
+ * by the new rows with the new tokens causal.  Both parts run on the paged attention kernel
+ * (mla_decode_paged): the new rows are presented to it as a pool of their own (copied to a
+ * 64-row-aligned layout in the workspace unless e is a multiple of 64), the prefix through a
+ * page table built from req_to_token.  The caller writes the new rows into the pool afterwards
+ * (mla_set_kv_buffer), as the page writes them after the two attention calls.
+ *   q                 bf16 [bs, e, h_q, 576]; e new tokens per request (uniform), h_q heads;
+ *                     e * h_q <= 65535 * 128
+ *   k_new             bf16 [bs, e, 576], 16-byte aligned: the new tokens' latent rows
+ *   kv_cache, kv_dtype, num_pages   the pool holding the prefix (bf16, e4m3 or e5m2, pages of
+ *                     64 rows), as for mla_decode_paged; descale_k with an fp8 pool
+ *   req_to_token .. rpi_dtype       the request-to-slot map, as for mla_build_block_table
+ *   prefix_lens       int32 [bs]: cached rows per request (0: no prefix; then o = o1)
+ *   max_prefix_pages  >= max cdiv(prefix_lens[b], 64) (longer prefixes are clamped and reported
+ *                     as by mla_build_block_table)
+ *   softmax_scale     applied to q . k
+ *   sm_count          SMs of the device (sizes the two split plans)
+ *   out, lse          bf16 [bs, e, h_q, 512] and fp32 [bs, e, h_q], written
+ *   workspace         at least mla_extend_workspace_bytes(bs, e, h_q, max_prefix_pages,
+ *                     sm_count) bytes, 256-byte aligned, zero-filled before its first use (the
+ *                     two attention calls' arrival words; every completed call leaves them zero)
+ * Errors: those of the calls it makes; MLA_ERR_WORKSPACE for a missing or short workspace.
+ */
+MLA_API mla_status_t mla_extend_paged_prefix(const void* q, int32_t bs, int32_t e, int32_t h_q, const void* k_new,
+                                             const void* kv_cache, int32_t kv_dtype, int64_t num_pages,
+                                             const int32_t* req_to_token, int64_t req_to_token_rows,
+                                             int64_t req_to_token_stride, const void* req_pool_indices,
+                                             int32_t rpi_dtype, const int32_t* prefix_lens, int32_t max_prefix_pages,
+                                             float softmax_scale, const float* descale_k, int32_t sm_count,
+                                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                             mla_stream_t stream);
+
+/*
  * Test hooks for the failure path of mla_decode_paged; not for production use.  They set
  * process-wide values that every later mla_decode_paged launch (from any thread) takes:
  *   wait_budget_ns  the budget of one pipeline wait (0 restores the default of 2 s);

@@ -83,6 +83,13 @@ def library() -> ctypes.CDLL:
     lib.mla_decode_paged.restype = I32
     lib.mla_set_kv_buffer.argtypes = [P, I32, I64, P, I32, I32, P, I64, P, P]
     lib.mla_set_kv_buffer.restype = I32
+    lib.mla_merge_state.argtypes = [P, P, P, P, I64, I32, P, P, P]
+    lib.mla_merge_state.restype = I32
+    lib.mla_extend_workspace_bytes.argtypes = [I32, I32, I32, I32, I32]
+    lib.mla_extend_workspace_bytes.restype = ctypes.c_size_t
+    lib.mla_extend_paged_prefix.argtypes = [P, I32, I32, I32, P, P, I32, I64, P, I64, I64, P, I32, P, I32,
+                                            ctypes.c_float, P, I32, P, P, P, ctypes.c_size_t, P]
+    lib.mla_extend_paged_prefix.restype = I32
     lib.mla_set_test_hooks.argtypes = [ctypes.c_uint64, I32]
     lib.mla_set_test_hooks.restype = I32
     lib.mla_read_device_error.argtypes = [ctypes.POINTER(I32), P]
@@ -319,6 +326,75 @@ def set_kv_buffer(k_cache: torch.Tensor, cache_loc: torch.Tensor, k: torch.Tenso
                                        _ptr(loc), _index_dtype(loc), n, _ptr(k), k.stride(0), _ptr(k_scale),
                                        _stream(k_cache.device)), "mla_set_kv_buffer")
     return k_cache
+
+
+def merge_state(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """merge_state(o1, s1, o2, s2) of two partial attention results of the same rows: bf16
+    o [..., 512] and fp32 natural-log lse [...] (-inf: no key).  Returns (o, lse)."""
+    _require_cuda(o_a, lse_a, o_b, lse_b, out, lse)
+    for o_, l_ in ((o_a, lse_a), (o_b, lse_b)):
+        if o_.dtype != torch.bfloat16 or not o_.is_contiguous() or o_.shape[-1] != 512:
+            raise ValueError("o must be a contiguous bf16 [..., 512] tensor")
+        if l_.dtype != torch.float32 or not l_.is_contiguous() or l_.numel() * 512 != o_.numel():
+            raise ValueError("lse must be a contiguous float32 tensor of one value per row")
+    if o_a.shape != o_b.shape:
+        raise ValueError("the two parts must have the same shape")
+    rows = lse_a.numel()
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse is None:
+        lse = torch.empty_like(lse_a)
+    _check(library().mla_merge_state(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), rows, 512, _ptr(out), _ptr(lse),
+                                     _stream(o_a.device)), "mla_merge_state")
+    return out, lse
+
+
+def extend_workspace_bytes(bs: int, e: int, h_q: int, max_prefix_pages: int, sm_count_: Optional[int] = None) -> int:
+    """Bytes of the extend workspace; allocate it zero-filled once and reuse it."""
+    return int(library().mla_extend_workspace_bytes(bs, e, h_q, max_prefix_pages,
+                                                    sm_count_ if sm_count_ is not None else sm_count()))
+
+
+def extend_paged_prefix(q: torch.Tensor, k_new: torch.Tensor, k_cache: torch.Tensor, req_to_token: torch.Tensor,
+                        req_pool_indices: torch.Tensor, prefix_lens: torch.Tensor, max_prefix_pages: int,
+                        softmax_scale: float, descale_k: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None):
+    """Extend with a cached prefix: q bf16 [bs, e, h_q, 576] of the e new tokens of every request
+    attends the new tokens' latent rows k_new (bf16 [bs, e, 576]) causally and the request's
+    prefix_lens[b] cached rows of k_cache (through req_to_token) in full; the two partial results
+    are merged by merge_state.  Returns (o bf16 [bs, e, h_q, 512], lse fp32 [bs, e, h_q])."""
+    _require_cuda(q, k_new, k_cache, req_to_token, req_pool_indices, prefix_lens, descale_k, out, lse, workspace)
+    if q.dim() != 4 or q.dtype != torch.bfloat16 or not q.is_contiguous() or q.shape[-1] != 576:
+        raise ValueError("q must be a contiguous bf16 [bs, e, h_q, 576] tensor")
+    bs, e, h_q, _ = (int(x) for x in q.shape)
+    if k_new.dtype != torch.bfloat16 or not k_new.is_contiguous() or tuple(k_new.shape) != (bs, e, 576):
+        raise ValueError("k_new must be a contiguous bf16 [bs, e, 576] tensor")
+    if k_cache.dtype not in _CACHE_DTYPES or not k_cache.is_contiguous() or k_cache.shape[-1] != 576:
+        raise ValueError("k_cache must be a contiguous bf16 / float8 pool with 576-wide rows")
+    if k_cache.numel() % (PAGE_SIZE * 576):
+        raise ValueError("k_cache must hold whole 64-token pages")
+    if req_to_token.dtype != torch.int32 or req_to_token.dim() != 2 or req_to_token.stride(1) != 1:
+        raise ValueError("req_to_token must be a row-major int32 matrix")
+    pl = prefix_lens.to(torch.int32).contiguous()
+    rpi = req_pool_indices.contiguous()
+    dev = q.device
+    if out is None:
+        out = torch.empty((bs, e, h_q, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((bs, e, h_q), dtype=torch.float32, device=dev)
+    need = extend_workspace_bytes(bs, e, h_q, int(max_prefix_pages)) if bs else 0
+    if workspace is None and need:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(library().mla_extend_paged_prefix(
+        _ptr(q), bs, e, h_q, _ptr(k_new), _ptr(k_cache), _CACHE_DTYPES[k_cache.dtype],
+        k_cache.numel() // (PAGE_SIZE * 576), _ptr(req_to_token), int(req_to_token.shape[0]),
+        req_to_token.stride(0), _ptr(rpi), _index_dtype(rpi), _ptr(pl), int(max_prefix_pages),
+        float(softmax_scale), _ptr(descale_k), sm_count(dev), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+        _stream(dev)), "mla_extend_paged_prefix")
+    return out, lse
 
 
 def set_test_hooks(wait_budget_ns: int = 0, withhold_tile: int = -1) -> None:

@@ -11,10 +11,13 @@
 #include <atomic>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/mla_b200.h"
 #include "block_table.cuh"
 #include "combine.cuh"
 #include "decode.cuh"
+#include "extend.cuh"
 #include "kv_write.cuh"
 #include "planner.cuh"
 
@@ -25,6 +28,13 @@ constexpr int kMaxDevices = 64;
 bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// An NVTX range around each entry point, named after it, for timeline tools (header-only NVTX:
+// without an attached tool a range costs a few nanoseconds).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so that the library
 // links against no driver library at build time and loads on hosts without a GPU.
@@ -107,6 +117,7 @@ mla_status_t mla_build_block_table(const int32_t* req_to_token, int64_t req_to_t
                                    int32_t seq_len_add, int32_t bs, int32_t* block_table,
                                    int64_t block_table_stride, int32_t max_pages,
                                    int32_t page_size, int32_t fill_tail, mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_build_block_table");
     if (bs < 0 || max_pages < 0 || page_size != 64) return MLA_ERR_INVALID_ARG;
     if (rpi_dtype != MLA_DTYPE_INT32 && rpi_dtype != MLA_DTYPE_INT64) return MLA_ERR_INVALID_ARG;
     if (seq_lens_dtype != MLA_DTYPE_INT32 && seq_lens_dtype != MLA_DTYPE_INT64)
@@ -143,6 +154,7 @@ mla_status_t mla_get_mla_metadata(const int32_t* cache_seqlens, int32_t bs,
                                   int32_t is_fp8_kvcache, int32_t sm_count,
                                   int32_t* tile_scheduler_metadata, int32_t* num_splits,
                                   mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_get_mla_metadata");
     (void)is_fp8_kvcache;  // accepted for call compatibility; the plan does not depend on it
     const int32_t num_sm_parts = mla_num_sm_parts(sm_count, num_heads_per_head_k, num_heads_k);
     if (bs < 0 || num_sm_parts < 1 || bs > (1 << 20)) return MLA_ERR_INVALID_ARG;
@@ -162,6 +174,7 @@ mla_status_t mla_build_decode_metadata(
     int32_t max_pages, int32_t page_size, int32_t fill_tail, int32_t num_heads_per_head_k,
     int32_t num_heads_k, int32_t is_fp8_kvcache, int32_t sm_count, int32_t* cache_seqlens,
     int32_t* tile_scheduler_metadata, int32_t* num_splits, mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_build_decode_metadata");
     (void)is_fp8_kvcache;  // accepted for call compatibility; the plan does not depend on it
     const int32_t parts = mla_num_sm_parts(sm_count, num_heads_per_head_k, num_heads_k);
     if (bs < 0 || max_pages < 0 || page_size != 64 || parts < 1 || bs > (1 << 20))
@@ -212,6 +225,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
                               int32_t causal, const float* descale_q, const float* descale_k,
                               void* out, float* lse, void* workspace, size_t workspace_bytes,
                               mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_decode_paged");
     if (bs < 0 || q_len <= 0 || h_q <= 0 || num_sm_parts < 1) return MLA_ERR_INVALID_ARG;
     if (head_dim != 576 || head_dim_v != 512 || page_size != 64) return MLA_ERR_UNSUPPORTED;
     if (q_dtype != MLA_DTYPE_BF16 && q_dtype != MLA_DTYPE_FP8_E4M3) return MLA_ERR_INVALID_ARG;
@@ -376,6 +390,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
 mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slots, const void* cache_loc,
                                int32_t loc_dtype, int32_t n_tokens, const void* k, int64_t k_row_stride,
                                const float* k_scale, mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_set_kv_buffer");
     if (n_tokens < 0 || num_slots < 0) return MLA_ERR_INVALID_ARG;
     if (kv_dtype != MLA_DTYPE_BF16 && kv_dtype != MLA_DTYPE_FP8_E4M3 && kv_dtype != MLA_DTYPE_FP8_E5M2)
         return MLA_ERR_INVALID_ARG;
@@ -402,6 +417,117 @@ mla_status_t mla_set_kv_buffer(void* kv_cache, int32_t kv_dtype, int64_t num_slo
     }
 #undef MLA_KV_LAUNCH
     return from_cuda(cudaGetLastError());
+}
+
+mla_status_t mla_merge_state(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                             int64_t rows, int32_t head_dim_v, void* o, float* lse, mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_merge_state");
+    if (rows < 0 || head_dim_v != 512) return rows < 0 ? MLA_ERR_INVALID_ARG : MLA_ERR_UNSUPPORTED;
+    if (rows == 0) return MLA_OK;
+    if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return MLA_ERR_INVALID_ARG;
+    if (!is_aligned(o_a, 16) || !is_aligned(o_b, 16) || !is_aligned(o, 16)) return MLA_ERR_INVALID_ARG;
+    const int64_t blocks = (rows + mla::kMergeStateWarps - 1) / mla::kMergeStateWarps;
+    if (blocks > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    mla::merge_state_kernel<<<(unsigned)blocks, mla::kMergeStateWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(o_a), lse_a, static_cast<const __nv_bfloat16*>(o_b), lse_b, rows,
+        static_cast<__nv_bfloat16*>(o), lse);
+    return from_cuda(cudaGetLastError());
+}
+
+namespace {
+// The extend workspace, 256-byte aligned parts in this order (sizes in bytes).
+struct ExtendLayout {
+    size_t pool, bt_r, cl_r, md_r, ns_r, ws_r, o1, lse1, bt_p, cl_p, md_p, ns_p, ws_p, o2, lse2, total;
+    int32_t parts, e_pad;
+    bool copy;
+};
+bool extend_layout(int32_t bs, int32_t e, int32_t h_q, int32_t max_prefix_pages, int32_t sm_count, ExtendLayout& L) {
+    if (bs <= 0 || e <= 0 || h_q <= 0 || max_prefix_pages < 0 || sm_count <= 0) return false;
+    L.parts = mla_num_sm_parts(sm_count, e * h_q, 1);
+    if (L.parts < 1) return false;
+    L.e_pad = (int32_t)(((int64_t)e + 63) / 64 * 64);
+    L.copy = L.e_pad != e;
+    const size_t rows = (size_t)bs * (size_t)e * (size_t)h_q;
+    const size_t ws = mla_decode_workspace_bytes(bs, e, h_q, L.parts);
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+    L.pool = take(L.copy ? (size_t)bs * L.e_pad * 576 * 2 : 0);
+    L.bt_r = take((size_t)bs * (L.e_pad / 64) * 4);
+    L.cl_r = take((size_t)bs * 4);
+    L.md_r = take((size_t)L.parts * 8 * 4);
+    L.ns_r = take(((size_t)bs + 1) * 4);
+    L.ws_r = take(ws);
+    L.o1 = take(rows * 512 * 2);
+    L.lse1 = take(rows * 4);
+    L.bt_p = take((size_t)bs * std::max(max_prefix_pages, 1) * 4);
+    L.cl_p = take((size_t)bs * 4);
+    L.md_p = take((size_t)L.parts * 8 * 4);
+    L.ns_p = take(((size_t)bs + 1) * 4);
+    L.ws_p = take(ws);
+    L.o2 = take(rows * 512 * 2);
+    L.lse2 = take(rows * 4);
+    L.total = off;
+    return true;
+}
+}  // namespace
+
+size_t mla_extend_workspace_bytes(int32_t bs, int32_t e, int32_t h_q, int32_t max_prefix_pages, int32_t sm_count) {
+    ExtendLayout L;
+    return extend_layout(bs, e, h_q, max_prefix_pages, sm_count, L) ? L.total : 0;
+}
+
+mla_status_t mla_extend_paged_prefix(const void* q, int32_t bs, int32_t e, int32_t h_q, const void* k_new,
+                                     const void* kv_cache, int32_t kv_dtype, int64_t num_pages,
+                                     const int32_t* req_to_token, int64_t req_to_token_rows,
+                                     int64_t req_to_token_stride, const void* req_pool_indices,
+                                     int32_t rpi_dtype, const int32_t* prefix_lens, int32_t max_prefix_pages,
+                                     float softmax_scale, const float* descale_k, int32_t sm_count, void* out,
+                                     float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+    const NvtxRange nvtx_range("mla_extend_paged_prefix");
+    if (bs == 0) return MLA_OK;
+    ExtendLayout L;
+    if (!extend_layout(bs, e, h_q, max_prefix_pages, sm_count, L)) return MLA_ERR_INVALID_ARG;
+    if ((int64_t)e * h_q > 65535LL * 128) return MLA_ERR_UNSUPPORTED;
+    if (!q || !k_new || !kv_cache || !prefix_lens || !out || !lse) return MLA_ERR_INVALID_ARG;
+    if (!is_aligned(k_new, 16)) return MLA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < L.total || !is_aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+    const int64_t ragged_pages = (int64_t)bs * (L.e_pad / 64);
+    if (ragged_pages * 64 > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+    auto i32 = [&](size_t off) { return reinterpret_cast<int32_t*>(w + off); };
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t rows = (size_t)bs * e * h_q;
+    mla_status_t r;
+    // (1) the new tokens among themselves, causal: their rows as a paged pool of their own
+    {
+        const int64_t units = L.copy ? (int64_t)bs * e * 72 : (int64_t)bs * (L.e_pad / 64);
+        const int64_t blocks = std::min<int64_t>((units + mla::kExtendThreads - 1) / mla::kExtendThreads, 4096);
+        mla::extend_ragged_view_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), mla::kExtendThreads, 0, st>>>(
+            static_cast<const uint4*>(k_new), bs, e, L.e_pad, L.copy ? static_cast<uint4*>(at(L.pool)) : nullptr,
+            i32(L.bt_r), i32(L.cl_r));
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+    r = mla_get_mla_metadata(i32(L.cl_r), bs, e * h_q, 1, 0, sm_count, i32(L.md_r), i32(L.ns_r), stream);
+    if (r != MLA_OK) return r;
+    r = mla_decode_paged(q, MLA_DTYPE_BF16, bs, e, h_q, 576, 512, L.copy ? at(L.pool) : k_new, MLA_DTYPE_BF16,
+                         ragged_pages, 64, i32(L.bt_r), L.e_pad / 64, L.e_pad / 64, i32(L.cl_r), i32(L.md_r), L.parts,
+                         i32(L.ns_r), softmax_scale, 1, nullptr, nullptr, at(L.o1),
+                         reinterpret_cast<float*>(at(L.lse1)), at(L.ws_r), L.o1 - L.ws_r, stream);
+    if (r != MLA_OK) return r;
+    // (2) the cached prefix, all of it
+    const int32_t mpp = std::max(max_prefix_pages, 1);
+    r = mla_build_decode_metadata(req_to_token, req_to_token_rows, req_to_token_stride, req_pool_indices, rpi_dtype,
+                                  prefix_lens, MLA_DTYPE_INT32, 0, bs, i32(L.bt_p), mpp, mpp, 64, 1, e * h_q, 1,
+                                  kv_dtype != MLA_DTYPE_BF16, sm_count, i32(L.cl_p), i32(L.md_p), i32(L.ns_p), stream);
+    if (r != MLA_OK) return r;
+    r = mla_decode_paged(q, MLA_DTYPE_BF16, bs, e, h_q, 576, 512, kv_cache, kv_dtype, num_pages, 64, i32(L.bt_p), mpp,
+                         mpp, i32(L.cl_p), i32(L.md_p), L.parts, i32(L.ns_p), softmax_scale, 0, nullptr, descale_k,
+                         at(L.o2), reinterpret_cast<float*>(at(L.lse2)), at(L.ws_p), L.o2 - L.ws_p, stream);
+    if (r != MLA_OK) return r;
+    // (3) merge_state
+    return mla_merge_state(at(L.o1), reinterpret_cast<const float*>(at(L.lse1)), at(L.o2),
+                           reinterpret_cast<const float*>(at(L.lse2)), (int64_t)rows, 512, out, lse, stream);
 }
 
 mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile) {

@@ -145,3 +145,55 @@ def test_block_table_and_planner_validation():
     assert dm(*{**okm, "md": (1 << 24) + 4}.values()) == 1
     assert dm(*{**okm, "r2t": None}.values()) == 1
     assert dm(*{**okm, "out_stride": 2}.values()) == 1
+
+
+def test_merge_state_validation():
+    lib = mla.library()
+    ms = lib.mla_merge_state
+    ok = dict(oa=1 << 20, la=1 << 21, ob=1 << 22, lb=1 << 23, rows=8, dv=512, o=1 << 24, lse=1 << 25, stream=None)
+    assert ms(*{**ok, "rows": 0}.values()) == 0              # nothing to merge
+    assert ms(*{**ok, "rows": -1}.values()) == 1
+    assert ms(*{**ok, "dv": 256}.values()) == 2
+    assert ms(*{**ok, "oa": None}.values()) == 1
+    assert ms(*{**ok, "lse": None}.values()) == 1
+    assert ms(*{**ok, "ob": (1 << 22) + 8}.values()) == 1   # misaligned o_b
+
+
+def test_extend_workspace_bytes():
+    """The extend workspace: a padded copy of the new rows (when e is not a multiple of 64),
+    then for each part a page table, lengths, plan, an attention workspace and the partial
+    result, every piece 256-byte aligned."""
+    lib = mla.library()
+    a256 = lambda x: -(-x // 256) * 256
+    for bs, e, h, mpp, sm in [(2, 37, 16, 4, 148), (3, 64, 128, 10, 148), (1, 1, 128, 0, 132)]:
+        parts = oracle.num_sm_parts(sm, e * h, 1)
+        e_pad = -(-e // 64) * 64
+        rows = bs * e * h
+        ws = lib.mla_decode_workspace_bytes(bs, e, h, parts)
+        pool = bs * e_pad * 576 * 2 if e_pad != e else 0
+        part = lambda pages: (a256(bs * pages * 4) + a256(bs * 4) + a256(parts * 32) + a256((bs + 1) * 4) + a256(ws)
+                              + a256(rows * 1024) + a256(rows * 4))
+        assert lib.mla_extend_workspace_bytes(bs, e, h, mpp, sm) == a256(pool) + part(e_pad // 64) + part(max(mpp, 1))
+    assert lib.mla_extend_workspace_bytes(0, 37, 16, 4, 148) == 0
+    assert lib.mla_extend_workspace_bytes(2, 0, 16, 4, 148) == 0
+    assert lib.mla_extend_workspace_bytes(2, 37, 16, -1, 148) == 0
+    assert lib.mla_extend_workspace_bytes(2, 37, 16, 4, 0) == 0
+
+
+def test_extend_validation_happens_before_any_launch():
+    lib = mla.library()
+    ex = lib.mla_extend_paged_prefix
+    ok = dict(q=1 << 20, bs=2, e=37, h=16, k_new=1 << 21, kv=1 << 22, kv_dt=0, pages=8, r2t=1 << 23, rows=5,
+              stride=512, rpi=1 << 24, rpi_dt=3, pl=1 << 25, mpp=4, scale=0.07, dk=None, sm=148, out=1 << 26,
+              lse=1 << 27, ws=1 << 28, ws_bytes=16, stream=None)
+    assert ex(*{**ok, "bs": 0}.values()) == 0                # idle batch
+    assert ex(*{**ok, "e": 0}.values()) == 1
+    assert ex(*{**ok, "h": 0}.values()) == 1
+    assert ex(*{**ok, "sm": 0}.values()) == 1
+    assert ex(*{**ok, "mpp": -1}.values()) == 1
+    assert ex(*{**ok, "q": None}.values()) == 1
+    assert ex(*{**ok, "pl": None}.values()) == 1
+    assert ex(*{**ok, "k_new": (1 << 21) + 8}.values()) == 1   # misaligned new rows
+    assert ex(*{**ok, "e": 65535, "h": 129}.values()) == 2     # more query rows than the kernel's grid holds
+    assert ex(*ok.values()) == 5                               # workspace too small
+    assert ex(*{**ok, "ws": None}.values()) == 5

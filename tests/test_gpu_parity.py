@@ -18,6 +18,10 @@ pytestmark = pytest.mark.gpu
 
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
+# Extend merges two bf16 partial results (each part's o is rounded to bf16, as the page's
+# merge_state receives them, then the merged o again): two roundings of outputs that stay
+# below 8 in magnitude are up to 2 x 2^-6 apart from one rounding, so the element bound doubles.
+EXTEND_MAX_ABS = 4e-2
 
 
 @pytest.fixture(scope="module")
@@ -52,7 +56,7 @@ def oracle_rows(wl, rows):
         q_is_fp8=wl.q_is_fp8)
 
 
-def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what="", max_abs=MAX_ABS):
     o_gpu = o_gpu.reshape(o_ref.shape)
     lse_gpu = lse_gpu.reshape(lse_ref.shape)
     dead = np.isneginf(lse_ref)
@@ -61,12 +65,12 @@ def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     live = ~dead
     assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
     err = np.abs(o_gpu - o_ref)
-    assert err.max() <= MAX_ABS, f"{what}: o max-abs {err.max():.3e}"
+    assert err.max() <= max_abs, f"{what}: o max-abs {err.max():.3e}"
     rel = np.linalg.norm(o_gpu - o_ref) / max(np.linalg.norm(o_ref), 1e-30)
     assert rel <= REL_L2, f"{what}: o rel-L2 {rel:.3e}"
     if live.any():
         lerr = np.abs(lse_gpu[live] - lse_ref[live])
-        assert lerr.max() <= MAX_ABS, f"{what}: lse max-abs {lerr.max():.3e}"
+        assert lerr.max() <= max_abs, f"{what}: lse max-abs {lerr.max():.3e}"
         lrel = np.linalg.norm(lse_gpu[live] - lse_ref[live]) / max(np.linalg.norm(lse_ref[live]), 1e-30)
         assert lrel <= REL_L2, f"{what}: lse rel-L2 {lrel:.3e}"
 
@@ -555,3 +559,86 @@ def test_unzeroed_workspace_is_reported(mla):
     ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
                                        wl.cache_seqlens, wl.softmax_scale, wl.causal)
     assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "after zero-fill")
+
+
+# ------------------------------------------------------------------ extend (prefix + new rows) and merge_state
+def test_merge_state_matches_oracle(mla):
+    """merge_state of two partial results against the oracle's log-sum-exp merge (rows where
+    one part, or both, saw no key included)."""
+    rng = np.random.default_rng(81)
+    rows = 300
+    oa = torch.from_numpy(rng.standard_normal((rows, 512)).astype(np.float32)).to(torch.bfloat16)
+    ob = torch.from_numpy(rng.standard_normal((rows, 512)).astype(np.float32)).to(torch.bfloat16)
+    la = rng.normal(0.0, 3.0, rows).astype(np.float32)
+    lb = rng.normal(0.0, 3.0, rows).astype(np.float32)
+    la[::7] = -np.inf
+    lb[::11] = -np.inf
+    o, lse = mla.merge_state(oa.cuda(), torch.from_numpy(la).cuda(), ob.cuda(), torch.from_numpy(lb).cuda())
+    torch.cuda.synchronize()
+    ref_o = np.zeros((rows, 512))
+    ref_lse = np.full((rows,), -np.inf)
+    a64, b64 = oa.double().numpy(), ob.double().numpy()
+    for r in range(rows):
+        if np.isneginf(la[r]) and np.isneginf(lb[r]):
+            continue
+        ref_o[r], ref_lse[r] = oracle.merge_states(np.stack([a64[r], b64[r]]), np.array([la[r], lb[r]]))
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "merge_state")
+
+
+def _new_rows(wl, prefix, e):
+    """The new tokens' latent rows: the last e positions of each request in the combined cache."""
+    pool = wl.kv_cache.reshape(-1, 576)
+    slots = torch.tensor([[int(wl.req_to_token[wl.req_pool_indices[b], prefix[b] + i]) for i in range(e)]
+                          for b in range(wl.bs)], dtype=torch.int64)
+    return pool[slots.reshape(-1)].reshape(wl.bs, e, 576).contiguous()
+
+
+@pytest.mark.parametrize("prefix,h,e", [([0, 130, 200, 64], 16, 37), ([300, 1, 0], 128, 64), ([513, 77], 40, 5),
+                                        ([2048, 700], 128, 130)])
+def test_extend_matches_attention_over_prefix_and_new_rows(mla, prefix, h, e):
+    """Extend as the FlashInfer backend page writes it (ragged causal part over the new rows, paged
+    part over the prefix, merge_state) against the oracle's single softmax over the prefix followed
+    by the new rows, the new tokens causal: the target-verify form of the same cache."""
+    wl = W.make_case(prefix, h=h, q_len=e, verify=True, seed=71 + e)
+    k_new = _new_rows(wl, prefix, e)
+    g = wl.to("cuda")
+    mpp = max(1, max(-(-p // 64) for p in prefix))
+    o, lse = mla.extend_paged_prefix(g.q, k_new.cuda(), g.kv_cache, g.req_to_token, g.req_pool_indices,
+                                     torch.tensor(prefix, dtype=torch.int32).cuda(), mpp, wl.softmax_scale)
+    torch.cuda.synchronize()
+    ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices, wl.cache_seqlens,
+                                       wl.softmax_scale, True)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, f"extend {prefix} h={h} e={e}",
+                 max_abs=EXTEND_MAX_ABS)
+    assert mla.read_device_error() == 0
+
+
+def test_extend_with_fp8_prefix(mla):
+    """An e4m3 prefix with its descale and bf16 new rows: the oracle computes the two parts on
+    their own (the ragged part over the new rows, causal; the paged part over the e4m3 prefix)
+    and merges them with its log-sum-exp merge."""
+    prefix, h, e = [150, 0, 64], 16, 9
+    wl = W.make_case(prefix, h=h, q_len=e, verify=True, kv="fp8", seed=91)
+    rng = np.random.default_rng(91)
+    k_new = torch.from_numpy(rng.standard_normal((wl.bs, e, 576)).astype(np.float32)).to(torch.bfloat16)
+    g = wl.to("cuda")
+    mpp = max(1, max(-(-p // 64) for p in prefix))
+    pl = torch.tensor(prefix, dtype=torch.int32)
+    o, lse = mla.extend_paged_prefix(g.q, k_new.cuda(), g.kv_cache, g.req_to_token, g.req_pool_indices, pl.cuda(),
+                                     mpp, wl.softmax_scale, descale_k=g.descale_k)
+    torch.cuda.synchronize()
+    dk = float(wl.descale_k[0])
+    o2, l2 = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices, pl.numpy(),
+                               wl.softmax_scale, False, kv_is_fp8=True, descale_k=dk)
+    r2t_new = np.arange(wl.bs * e, dtype=np.int32).reshape(wl.bs, e)
+    o1, l1 = oracle.mla_decode(wl.q, k_new.reshape(-1, 576), r2t_new, np.arange(wl.bs), np.full(wl.bs, e, np.int32),
+                               wl.softmax_scale, True)
+    ref_o = np.zeros_like(o1)
+    ref_lse = np.full(l1.shape, -np.inf)
+    for idx in np.ndindex(l1.shape):
+        if np.isneginf(l1[idx]) and np.isneginf(l2[idx]):
+            continue
+        ref_o[idx], ref_lse[idx] = oracle.merge_states(np.stack([o1[idx], o2[idx]]), np.array([l1[idx], l2[idx]]))
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "extend, e4m3 prefix",
+                 max_abs=EXTEND_MAX_ABS)
+    assert mla.read_device_error() == 0
