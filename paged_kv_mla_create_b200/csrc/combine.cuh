@@ -158,15 +158,24 @@ __device__ __forceinline__ bool merge_rows_cta_bulk(const float* __restrict__ pa
 }
 
 // The rows of requests of more than kFusedMergeMaxPieces pieces (the others were written whole or
-// merged by the attention kernel, so the launch needs no host knowledge of the plan): each warp
-// takes (request, query row) pairs in turn, a grid of about one CTA per SM, so that a batch
-// with nothing left to merge costs one pass over the plan rather than a CTA per 8 rows.
+// merged by the attention kernel, so the launch needs no host knowledge of the plan): each CTA
+// first stages num_splits in shared memory (one coalesced read, for up to kCombineStagedRequests
+// requests), then its warps take (request, query row) pairs in turn; a grid of about one CTA per
+// SM, so that a batch with nothing left to merge costs one pass over the plan.
+constexpr int kCombineStagedRequests = 4096;
+
 __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                       const int32_t* __restrict__ num_splits, int32_t rows, int32_t bs,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+    __shared__ int32_t s_ns[kCombineStagedRequests + 1];
     // launched as a programmatic dependent of the attention kernel: wait for all of it
     pdl_wait_prerequisites();
+    const bool staged = bs <= kCombineStagedRequests;
+    if (staged) {
+        for (int b = threadIdx.x; b <= bs; b += blockDim.x) s_ns[b] = num_splits[b];
+        __syncthreads();
+    }
     const uint64_t read_pol = l2_policy_evict_first();   // the partials are read once
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * kCombineWarps;
@@ -174,8 +183,8 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
     for (int64_t idx = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5); idx < total; idx += warps) {
         const int b = (int)(idx / rows);
         const int row = (int)(idx - (int64_t)b * rows);
-        const int s0 = num_splits[b];
-        const int n = num_splits[b + 1] - s0;
+        const int s0 = staged ? s_ns[b] : num_splits[b];
+        const int n = (staged ? s_ns[b + 1] : num_splits[b + 1]) - s0;
         if (n <= kFusedMergeMaxPieces) continue;
         const int64_t out_row = (int64_t)b * rows + row;
         merge_row(part_o, part_lse, s0, n, rows, row, out + out_row * 512, lse_out + out_row, lane, read_pol);
