@@ -124,10 +124,14 @@ enum : int {
 // of split requests, and the fold decision of the current epilogue.
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kMiscFold = 8;          // int index into the misc area: the fold-in decision
-// Fold-in merge: the other piece's partial rows, copied into the idle K ring one 2 KB row per
-// copy at this stride (16 bytes of padding rotate the rows' banks).
-constexpr int kFoldRowStride = kDv * 4 + 16;
-static_assert(kCtaRows * kFoldRowStride <= kKSlots * kKSlotBytes, "fold-in rows fit the K ring");
+// Fold-in merge: the other piece's 64 partial rows land in the idle K ring as sixteen 2-D TMA
+// boxes of 32 fp32 columns x 64 rows (8 KB each, 128-byte swizzle: 16-byte unit u of row r at
+// u ^ (r & 7), so that the row-per-lane reads are conflict-free).  Sixteen loads, not one per row:
+// a TMA operation costs ~70 cycles of the SM's TMA unit whatever its size.
+constexpr int kFoldBoxCols = 32;
+constexpr int kFoldBoxBytes = kCtaRows * kFoldBoxCols * 4;   // 8 KB
+constexpr int kFoldBoxes = kDv / kFoldBoxCols;               // 16
+static_assert(kFoldBoxes * kFoldBoxBytes <= kKSlots * kKSlotBytes, "fold-in rows fit the K ring");
 constexpr int kMaxPendingMerges = 2;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -227,6 +231,7 @@ struct Params {
     int32_t* arrivals;             // [bs, query tiles, 2]: split pieces arrived (zero between calls)
     uint64_t wait_budget_ns;       // budget of one pipeline wait
     int32_t withhold_tile;         // test hook: the leader's K load of this tile is not issued (-1: none)
+    int32_t fold_ok;               // po_map covers part_o (else no fold-in merge)
 };
 
 // The work units of a part, identical in every role: request b, block range [kb0, kb1).
@@ -313,7 +318,8 @@ struct PageWindow {
 template <int kKv, bool kFp8Q>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
-                  const __grid_constant__ CUtensorMap q_map, const __grid_constant__ Params p) {
+                  const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap po_map,
+                  const __grid_constant__ Params p) {
     constexpr bool kFp8 = kKv != 0;
     constexpr bool kE5M2 = kKv == 2;
     static_assert(kKv == 1 || !kFp8Q, "e4m3 queries need an e4m3 cache");
@@ -387,6 +393,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         prefetch_tensormap(&k_map);
         prefetch_tensormap(&v_map);
         prefetch_tensormap(&q_map);
+        prefetch_tensormap(&po_map);
     }
     tc_fence_before();
     __syncthreads();
@@ -974,7 +981,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             // its own O and writes the final o; it stores no partial of its own.
             int32_t* const arrival = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
             if (t == 0)
-                pending[kMiscFold] = (!direct && pieces == 2 && pieces <= kFusedMergeMaxPieces && last_unit &&
+                pending[kMiscFold] = (p.fold_ok && !direct && pieces == 2 && pieces <= kFusedMergeMaxPieces && last_unit &&
                                      ld_acquire_gpu(arrival) == 1) ? 1 : 0;
             xmax[256 + t] = l_half;
             mbar_arrive(bar(kBarLx));
@@ -989,13 +996,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 const int other = s0 + 1 - (split - s0);
                 const int row_base = mtile * kRows + kCtaRows * (int)rank;
                 const int nrows = min(kCtaRows, p.rows - row_base);
-                if (warp == kSoftmaxWarp0) {
-                    if (lane == 0) mbar_arrive_expect_tx(bar(kBarFold), (uint32_t)nrows * (kDv * 4));
+                if (warp == kSoftmaxWarp0 && lane == 0) {
+                    // rows past this CTA's last (a partial query tile) read the next piece's rows, or
+                    // zeros past the workspace: loaded, never used
+                    (void)nrows;
+                    mbar_arrive_expect_tx(bar(kBarFold), (uint32_t)(kFoldBoxes * kFoldBoxBytes));
                     fence_proxy_async_global();   // the acquired partial rows, read by the async proxy
-                    __syncwarp();
-                    for (int r = lane; r < nrows; r += 32)
-                        bulk_load(sbase + kOffK + (uint32_t)(r * kFoldRowStride),
-                                  p.part_o + ((int64_t)other * p.rows + row_base + r) * kDv, kDv * 4, bar(kBarFold));
+#pragma unroll 1
+                    for (int j = 0; j < kFoldBoxes; ++j)
+                        tma_load_2d(sbase + kOffK + (uint32_t)(j * kFoldBoxBytes), &po_map, bar(kBarFold),
+                                    kFoldBoxCols * j, other * p.rows + row_base);
                 }
                 // merged lse and the two weights (log2 units): own (m_run, l_run), other lse_o
                 const float lse_o = row_valid ? __ldcg(p.part_lse + (int64_t)other * p.rows + rowg) : -INFINITY;
@@ -1043,10 +1053,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         if (fold) {
                             // own O (normalised and weighted) + the other piece's row, weighted
                             col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
-                            const uint32_t orow = sbase + kOffK + (uint32_t)(rloc * kFoldRowStride + col * 4);
+                            // columns col .. col + 63: boxes col / 32 and the next, 16-byte units
+                            // k / 2 = 8 (box) + u at u ^ (rloc & 7) in row rloc of its box
+                            const uint32_t orow = sbase + kOffK + (uint32_t)((col / kFoldBoxCols) * kFoldBoxBytes + rloc * 128);
 #pragma unroll
                             for (int k = 0; k < 32; k += 2) {
-                                const uint4 v = ld_shared_v4u(orow + 8u * (uint32_t)k);
+                                const uint32_t f4 = (uint32_t)(k >> 1);   // float4 index 0 .. 15
+                                const uint4 v = ld_shared_v4u(orow + (f4 >> 3) * (uint32_t)kFoldBoxBytes +
+                                                              (((f4 & 7u) ^ (uint32_t)(rloc & 7)) << 4));
                                 w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv + __uint_as_float(v.x) * other_w,
                                                    __uint_as_float(raw[2 * k + 1]) * inv + __uint_as_float(v.y) * other_w);
                                 w[k + 1] = pack_bf16x2(__uint_as_float(raw[2 * k + 2]) * inv + __uint_as_float(v.z) * other_w,

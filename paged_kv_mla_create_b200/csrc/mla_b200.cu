@@ -351,19 +351,34 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     p.part_o = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q));
     p.part_lse = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q) +
                                           align256(splits * rows * 512 * sizeof(float)));
+    // part_o as a 2-D fp32 tensor (512 columns [2048 B], splits * rows rows) for the fold-in
+    // merge's loads: boxes of 32 columns x 64 rows, 128-byte swizzle
+    CUtensorMap po_map;
+    std::memset(&po_map, 0, sizeof po_map);
+    p.fold_ok = 0;
+    if ((uint64_t)splits * (uint64_t)rows <= (uint64_t)INT32_MAX) {
+        const cuuint64_t gdim[2] = {512, (cuuint64_t)splits * (cuuint64_t)rows};
+        const cuuint64_t gstride[1] = {512 * sizeof(float)};
+        const cuuint32_t box[2] = {(cuuint32_t)mla::decode::kFoldBoxCols, (cuuint32_t)mla::decode::kCtaRows};
+        const cuuint32_t estride[2] = {1, 1};
+        if (encode(&po_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.part_o, gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            p.fold_ok = 1;
+    }
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
     using mla::decode::kSmemBytes;
     using mla::decode::kThreads;
     if (q_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E5M2)
-        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
     else
-        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, p);
+        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
