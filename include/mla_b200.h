@@ -358,13 +358,16 @@ MLA_API mla_status_t mla_extend_paged_prefix(const void* q, int32_t bs, int32_t 
  *   wait_budget_ns  the budget of one pipeline wait (0 restores the default of 2 s);
  *   withhold_tile   the index (within a scheduler part, counting from 0) of a tile whose page
  *                   load the leader CTA of every pair does not issue, so that the wait for it
- *                   runs out (-1 restores normal operation).
+ *                   runs out (-1 restores normal operation);
+ *   no_fold_in      nonzero: the last piece of a split request never folds the other pieces
+ *                   into its own result but stores its partial and merges at the end of its
+ *                   part (the two ways give identical bits; 0 restores normal operation).
  * When a wait runs out the CTA records MLA_DEVERR_WAIT_TIMEOUT, both CTAs of the pair stop at
  * their next wait, let their issued copies land, release their tensor memory and return; the
  * call's outputs are then undefined and its workspace must be zero-filled again.  Host-only,
  * no synchronisation.  Returns MLA_ERR_INVALID_ARG for withhold_tile < -1.
  */
-MLA_API mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile);
+MLA_API mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile, int32_t no_fold_in);
 
 /*
  * Read and clear the sticky device error word of the current device (a bitwise OR of

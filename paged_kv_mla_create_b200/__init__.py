@@ -90,7 +90,7 @@ def library() -> ctypes.CDLL:
     lib.mla_extend_paged_prefix.argtypes = [P, I32, I32, I32, P, P, I32, I64, P, I64, I64, P, I32, P, I32,
                                             ctypes.c_float, P, I32, P, P, P, ctypes.c_size_t, P]
     lib.mla_extend_paged_prefix.restype = I32
-    lib.mla_set_test_hooks.argtypes = [ctypes.c_uint64, I32]
+    lib.mla_set_test_hooks.argtypes = [ctypes.c_uint64, I32, I32]
     lib.mla_set_test_hooks.restype = I32
     lib.mla_read_device_error.argtypes = [ctypes.POINTER(I32), P]
     lib.mla_read_device_error.restype = I32
@@ -397,10 +397,13 @@ def extend_paged_prefix(q: torch.Tensor, k_new: torch.Tensor, k_cache: torch.Ten
     return out, lse
 
 
-def set_test_hooks(wait_budget_ns: int = 0, withhold_tile: int = -1) -> None:
-    """Test-only: the pipeline wait budget (0: the default 2 s) and a tile whose page load the
-    leader CTAs withhold (-1: none) for every later attention launch in this process."""
-    _check(library().mla_set_test_hooks(int(wait_budget_ns), int(withhold_tile)), "mla_set_test_hooks")
+def set_test_hooks(wait_budget_ns: int = 0, withhold_tile: int = -1, no_fold_in: bool = False) -> None:
+    """Test-only: the pipeline wait budget (0: the default 2 s), a tile whose page load the
+    leader CTAs withhold (-1: none) and whether the last piece of a split request must merge by
+    stored partials instead of folding the others in, for every later attention launch in this
+    process."""
+    _check(library().mla_set_test_hooks(int(wait_budget_ns), int(withhold_tile), int(bool(no_fold_in))),
+           "mla_set_test_hooks")
 
 
 def read_device_error(device=None) -> int:

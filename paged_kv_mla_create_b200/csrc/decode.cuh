@@ -39,12 +39,17 @@
 //     can never strand the others), P goes to shared memory for the PV MMA, O is rescaled
 //     in tensor memory only when the running maximum grows by more than 2^8, and the
 //     epilogue normalises and writes o and lse.
-//   * A unit whose block range is a whole request writes bf16 o and lse directly; a split
-//     piece writes fp32 partials, then counts its arrival on a per-(request, query tile,
-//     CTA) word of the workspace.  For a request of at most kFusedMergeMaxPieces pieces the
-//     CTA whose arrival completes the count merges the pieces' partials of its 64 rows
-//     (log-sum-exp) once its part is done, with all its warps, and resets the word to zero;
-//     combine_splits_kernel merges requests of more pieces.
+//   * A unit whose block range is a whole request writes bf16 o and lse directly.  A piece of a
+//     request of at most kFusedMergeMaxPieces pieces claims a place on a per-(request, query
+//     tile, CTA) word of the workspace during its last tile; the last to claim merges the
+//     request's rows (log-sum-exp), the others store fp32 partials and count them stored on
+//     the same word.  The last claimer, if in its part's last unit (Q, K ring and P idle) and
+//     the request has at most kFoldMaxPieces pieces, folds the others' stored rows into its own
+//     tensor-memory O in the epilogue (waiting for their stores if need be); otherwise it stores
+//     its partial too and merges all of them once its part is done.  Both ways sum the pieces
+//     in split-slot order with the same weights, so the result has the same bits whichever
+//     piece merges.  The merging CTA resets the word to zero; combine_splits_kernel merges
+//     requests of more pieces.
 //   * e4m3 queries with an e4m3 cache (the backend page's fp8 recipe: q quantised with the
 //     cache's scale, descale_q and descale_k passed along): S runs as kind::f8f6f4 MMAs (K = 32
 //     per instruction, 18 per tile) straight from the raw page and the e4m3 query rows, both in a
@@ -113,7 +118,9 @@ enum : int {
     kBarLx = kBarXchg + 2,              // local: the 128 softmax threads posted row sums
     kBarPartial,                        // local: the 128 softmax threads stored a split piece
     kBarVWiden,                         // local, e4m3 q: warps 8..11 read their raw V chunks
-    kBarFold,                           // local: the other piece's partial rows landed (fold-in merge)
+    kBarFold,                           // local: the other pieces' partial rows landed (fold-in merge)
+    kBarFoldRd,                         // local: the 128 softmax threads read the first fold-in round
+    kBarFoldL,                          // local: the other pieces' lse values landed (fold-in merge)
     kBarMerge,                          // local: a tail merge's pass of partial rows landed
     kBarKRaw,                           // local (x2), e4m3 cache: this CTA's page landed
     kNumBars = kBarKRaw + kKSlots
@@ -124,14 +131,25 @@ enum : int {
 // of split requests, and the fold decision of the current epilogue.
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kMiscFold = 8;          // int index into the misc area: the fold-in decision
-// Fold-in merge: the other piece's 64 partial rows land in the idle K ring as sixteen 2-D TMA
-// boxes of 32 fp32 columns x 64 rows (8 KB each, 128-byte swizzle: 16-byte unit u of row r at
-// u ^ (r & 7), so that the row-per-lane reads are conflict-free).  Sixteen loads, not one per row:
-// a TMA operation costs ~70 cycles of the SM's TMA unit whatever its size.
+// Fold-in merge: the other pieces' 64 partial rows land in the idle Q, K ring and P areas
+// (contiguous from the base, 200 KB) as 2-D TMA boxes of 32 fp32 columns x 64 rows (8 KB each,
+// 128-byte swizzle: 16-byte unit u of row r at u ^ (r & 7), so that the row-per-lane reads are
+// conflict-free); a TMA operation costs ~70 cycles of the SM's TMA unit whatever its size, so
+// boxes, not rows.  One other piece: all sixteen boxes at once, box c at 8 KB * c.  Two or three:
+// the eight boxes of columns [0, 256) of every other piece j at 8 KB * (8 j + c), then, once those
+// are read, the eight of columns [256, 512) in the same places.
 constexpr int kFoldBoxCols = 32;
 constexpr int kFoldBoxBytes = kCtaRows * kFoldBoxCols * 4;   // 8 KB
 constexpr int kFoldBoxes = kDv / kFoldBoxCols;               // 16
-static_assert(kFoldBoxes * kFoldBoxBytes <= kKSlots * kKSlotBytes, "fold-in rows fit the K ring");
+// Requests of up to this many pieces fold in (four-piece requests merge at the end of the part:
+// the fold's unrolled sums over four pieces exceed the register budget).
+constexpr int kFoldMaxPieces = 3;
+static_assert(kOffQ == 0 && kOffK == kOffQ + kQHiBytes && kOffP == kOffK + kKSlots * kKSlotBytes,
+              "the fold-in staging is contiguous");
+static_assert(kFoldBoxes * kFoldBoxBytes <= kOffX - kOffQ &&
+                  (kFoldMaxPieces - 1) * (kFoldBoxes / 2) * kFoldBoxBytes <= kOffX - kOffQ &&
+                  kFoldMaxPieces <= kFusedMergeMaxPieces,
+              "fold-in rows fit the idle areas");
 constexpr int kMaxPendingMerges = 2;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -231,7 +249,7 @@ struct Params {
     int32_t* arrivals;             // [bs, query tiles, 2]: split pieces arrived (zero between calls)
     uint64_t wait_budget_ns;       // budget of one pipeline wait
     int32_t withhold_tile;         // test hook: the leader's K load of this tile is not issued (-1: none)
-    int32_t fold_ok;               // po_map covers part_o (else no fold-in merge)
+    int32_t fold_ok;               // po_map / pl_map cover part_o / part_lse (else no fold-in merge)
 };
 
 // The work units of a part, identical in every role: request b, block range [kb0, kb1).
@@ -278,6 +296,59 @@ __device__ __forceinline__ UnitIter make_iter(const Params& p, int part, bool& o
 
 __device__ __forceinline__ int tiles_of(int kb0, int kb1) { return (kb1 - kb0 + 1) >> 1; }
 
+// A split request's arrival word (per query tile and CTA): its low 16 bits count the pieces that
+// claimed a place (the last to claim merges), its high bits the pieces that stored their partial
+// rows.  Bounded wait until `target` pieces have stored theirs.  Only pieces that have already
+// claimed are waited for, and a piece stores right after it claims without waiting on any other
+// CTA, so the wait ends unless a piece gave up (abort).
+__device__ __forceinline__ bool wait_stored(const int32_t* word, int target, const AbortCtl& a) {
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if ((ld_acquire_gpu(word) >> 16) >= target) return true;
+        if (*a.flag) return false;
+        if (global_timer_ns() - t0 > a.budget_ns) {
+            raise_abort(a);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+// One 64-column step of the fold-in merge for one row (NP pieces, this one in slot OWN): for each
+// 16-byte group of 4 columns, the
+// pieces' rows in split-slot order, weighted and summed (acc += w_i * v_i from zero, exactly as
+// the merge of stored partials computes it), then packed to bf16.  This piece's own row is its
+// tensor-memory O times inv (its stored partial's value), the others' (NP - 1 of them) come from
+// the staged boxes at base_j + off(group).  Branch-free, so that the shared-memory loads of four
+// groups can be issued ahead of their sums.
+template <int NP, int OWN>
+__device__ __forceinline__ void fold_step(const uint32_t (&raw)[64], uint32_t (&w)[32], float inv, const float* wts,
+                                          uint32_t base0, uint32_t base1, int rloc) {
+    const uint32_t row = (uint32_t)rloc * 128u, sw = (uint32_t)rloc & 7u;
+#pragma unroll
+    for (int f4 = 0; f4 < 16; ++f4) {
+        const uint32_t off = (uint32_t)(f4 >> 3) * (uint32_t)kFoldBoxBytes + row + ((((uint32_t)f4 & 7u) ^ sw) << 4);
+        float4 o[NP - 1];
+        o[0] = ld_shared_v4f(base0 + off);
+        if constexpr (NP > 2) o[NP - 2] = ld_shared_v4f(base1 + off);
+        const float4 mine = make_float4(__uint_as_float(raw[4 * f4]) * inv, __uint_as_float(raw[4 * f4 + 1]) * inv,
+                                        __uint_as_float(raw[4 * f4 + 2]) * inv, __uint_as_float(raw[4 * f4 + 3]) * inv);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+            // slot i: this piece, or the other piece j = i - 1 (i > OWN) / j = i (i < OWN)
+            const float4 v = i == OWN ? mine : o[i > OWN ? (i > 0 ? i - 1 : 0) : (i < NP - 1 ? i : NP - 2)];
+            acc.x += wts[i] * v.x;
+            acc.y += wts[i] * v.y;
+            acc.z += wts[i] * v.z;
+            acc.w += wts[i] * v.w;
+        }
+        w[2 * f4] = pack_bf16x2(acc.x, acc.y);
+        w[2 * f4 + 1] = pack_bf16x2(acc.z, acc.w);
+        if ((f4 & 3) == 3) __syncwarp();   // loads hoisted four groups ahead at most (registers)
+    }
+}
+
 // Page ids of one unit's blocks for a whole warp: lanes hold blocks [base, base + 32), slid
 // forward as the tiles advance.  row(blk) is the TMA row coordinate page * 64, or the first
 // row past the pool (read as zeros) for a block past the unit or a bad page id.
@@ -319,7 +390,7 @@ template <int kKv, bool kFp8Q>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
                   const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap po_map,
-                  const __grid_constant__ Params p) {
+                  const __grid_constant__ CUtensorMap pl_map, const __grid_constant__ Params p) {
     constexpr bool kFp8 = kKv != 0;
     constexpr bool kE5M2 = kKv == 2;
     static_assert(kKv == 1 || !kFp8Q, "e4m3 queries need an e4m3 cache");
@@ -367,6 +438,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         mbar_init(bar(kBarQFull), kFp8Q ? 1 : (kFp8 ? 0 : 1) + 4);
         mbar_init(bar(kBarVWiden), 128);
         mbar_init(bar(kBarFold), 1);
+        mbar_init(bar(kBarFoldRd), 128);
+        mbar_init(bar(kBarFoldL), 1);
         mbar_init(bar(kBarMerge), 1);
         mbar_init(bar(kBarQEmpty), 1);
         for (int j = 0; j < 2; ++j) {
@@ -394,6 +467,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         prefetch_tensormap(&v_map);
         prefetch_tensormap(&q_map);
         prefetch_tensormap(&po_map);
+        prefetch_tensormap(&pl_map);
     }
     tc_fence_before();
     __syncthreads();
@@ -856,6 +930,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             if (lim > L) lim = L;
             if (lim > kb1 * kPage) lim = kb1 * kPage;   // keys of this unit only
             float m_run = -INFINITY, l_half = 0.f;
+            // A piece of a request merged in this kernel claims its place once the last tile's P is
+            // written, so that the atomic's round trip overlaps the last PV (acquire: a claim that
+            // finds every other piece stored also sees their rows).
+            int32_t* const arrival = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
+            const bool merged_here = !direct && pieces <= kFusedMergeMaxPieces;
+            int claim_old = 0;
             for (int i = 0; i < n; ++i, ++g) {
                 const uint32_t sb = g & 1u;
                 if (!mbar_wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, actl)) {
@@ -971,60 +1051,103 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         st_async_b32(map_to_cta(sbase + kOffPSig + 4u * (uint32_t)(warp - kSoftmaxWarp0), 0), g,
                                      map_to_cta(bar(kBarPFull), 0));
                 }
+                if (t == 0 && merged_here && i == n - 1) claim_old = atom_add_acquire_gpu(arrival, 1);
             }
             if (!alive) break;
             // epilogue of the unit
             if (!mbar_wait_bounded(bar(kBarOFull), uq & 1u, actl)) break;
             tc_fence_after();
-            // Fold-in merge: a piece of a two-piece request, in its part's last unit (the K ring
-            // is idle), whose other piece has already stored its partial rows, merges them into
-            // its own O and writes the final o; it stores no partial of its own.
-            int32_t* const arrival = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
-            if (t == 0)
-                pending[kMiscFold] = (p.fold_ok && !direct && pieces == 2 && pieces <= kFusedMergeMaxPieces && last_unit &&
-                                     ld_acquire_gpu(arrival) == 1) ? 1 : 0;
+            // How this piece ends (t == 0 decides from its claim): 0 whole request (or a piece of
+            // one merged by the merge kernel), 1 store the partial rows and count them, 2 the last
+            // claimer in its part's last unit (Q, K ring and P idle): fold the other pieces' rows
+            // into its own O and write the final o, 3 the last claimer elsewhere: store, then merge
+            // at the end of the part.
+            if (t == 0) {
+                int mode = 0;
+                if (merged_here) {
+                    const int claimed = claim_old & 0xFFFF, stored = (claim_old >> 16) & 0x7FFF;
+                    mode = 1;
+                    if (claim_old < 0 || claimed >= pieces || stored > claimed)
+                        raise_error(128 /* MLA_DEVERR_WORKSPACE_STATE */);
+                    else if (claimed == pieces - 1)
+                        mode = (p.fold_ok && last_unit && pieces <= kFoldMaxPieces) ? 2 : 3;
+                }
+                pending[kMiscFold] = mode;
+            }
             xmax[256 + t] = l_half;
             mbar_arrive(bar(kBarLx));
             if (!mbar_wait_bounded(bar(kBarLx), uq & 1u, actl)) break;
-            const bool fold = pending[kMiscFold] != 0;
+            const int mode = pending[kMiscFold];
+            const bool fold = mode == 2;
             const float l_run = l_half + xmax[256 + (t ^ 64)];
-            float inv = l_run > 0.f ? dk / l_run : 0.f;
+            // the partial state in the stored form (also the fold's own piece)
+            const float inv = l_run > 0.f ? dk / l_run : 0.f;
             float lse_val = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-            float other_w = 0.f;
-            if (fold) {
-                const int s0 = p.num_splits[ub];
-                const int other = s0 + 1 - (split - s0);
-                const int row_base = mtile * kRows + kCtaRows * (int)rank;
-                const int nrows = min(kCtaRows, p.rows - row_base);
-                if (warp == kSoftmaxWarp0 && lane == 0) {
-                    // rows past this CTA's last (a partial query tile) read the next piece's rows, or
-                    // zeros past the workspace: loaded, never used
-                    (void)nrows;
-                    mbar_arrive_expect_tx(bar(kBarFold), (uint32_t)(kFoldBoxes * kFoldBoxBytes));
-                    fence_proxy_async_global();   // the acquired partial rows, read by the async proxy
+            // fold-in: the pieces' weights in split-slot order, as the merge of stored partials
+            // computes them (so that the result does not depend on which piece merges)
+            float wts[kFoldMaxPieces];
+            // this piece's index in the request (nonzero only for a part's first unit) and the
+            // request's first split slot, read only where a merge needs them
+            const int own = (mode >= 2 && ub == iter.first_b) ? p.md[8 * part + 4] : 0;
+            const int s0 = split - own;
+            const int row_base = mtile * kRows + kCtaRows * (int)rank;
+            // rows past this CTA's last (a partial query tile) load the next piece's rows, or
+            // zeros past the workspace: loaded, never used
+            // (one TMA operation brings eight boxes; in the first round the other pieces' 64 lse
+            // values come too, into the row-max exchange area, idle now: piece j at 256 j bytes)
+            auto fold_issue = [&](int round) {
+                const int nbox = pieces == 2 ? kFoldBoxes : kFoldBoxes / 2;
+                if (round == 0) mbar_arrive_expect_tx(bar(kBarFoldL), (uint32_t)((pieces - 1) * kCtaRows * 4));
+                mbar_arrive_expect_tx(bar(kBarFold), (uint32_t)((pieces - 1) * nbox * kFoldBoxBytes));
 #pragma unroll 1
-                    for (int j = 0; j < kFoldBoxes; ++j)
-                        tma_load_2d(sbase + kOffK + (uint32_t)(j * kFoldBoxBytes), &po_map, bar(kBarFold),
-                                    kFoldBoxCols * j, other * p.rows + row_base);
+                for (int j = 0; j < pieces - 1; ++j) {
+                    const int slot = s0 + j + (j >= own ? 1 : 0);
+                    if (round == 0)
+                        tma_load_2d(sbase + kOffX + 256u * (uint32_t)j, &pl_map, bar(kBarFoldL), row_base, slot);
+#pragma unroll 1
+                    for (int c = 0; c < nbox; c += 8)
+                        tma_load_3d(sbase + kOffQ + (uint32_t)((pieces == 2 ? c : 8 * j + c) * kFoldBoxBytes), &po_map,
+                                    bar(kBarFold), 0, slot * p.rows + row_base, 8 * round + c);
                 }
-                // merged lse and the two weights (log2 units): own (m_run, l_run), other lse_o
-                const float lse_o = row_valid ? __ldcg(p.part_lse + (int64_t)other * p.rows + rowg) : -INFINITY;
-                const float own2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
-                const float oth2 = lse_o * 1.4426950408889634f;
-                const float mx = fmaxf(own2, oth2);
-                if (mx == -INFINITY) {
-                    inv = 0.f;
+            };
+            if (fold) {
+                if (t == 0) {
+                    // the others have claimed before this piece: unless the claim found them all
+                    // stored, wait until they have
+                    if (((claim_old >> 16) & 0x7FFF) >= pieces - 1 || wait_stored(arrival, pieces - 1, actl)) {
+                        *arrival = 0;   // every piece is done with the word: ready for the next call
+                        fence_proxy_async_global();   // the acquired partial rows, read by the async proxy
+                        fence_proxy_async_smem();     // the exchange area, written by the async proxy
+                        fold_issue(0);
+                    }
+                }
+                // the weights while the rows are in flight (one fold per CTA at most: phase 0)
+                if (!mbar_wait_bounded(bar(kBarFoldL), 0u, actl)) break;
+                float m = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < kFoldMaxPieces; ++i) {
+                    wts[i] = -INFINITY;
+                    if (i < pieces)
+                        wts[i] = i == own ? lse_val : (row_valid ? xmax[64 * (i - (i > own ? 1 : 0)) + rloc] : -INFINITY);
+                    m = fmaxf(m, wts[i]);
+                }
+                if (m == -INFINITY) {
+#pragma unroll
+                    for (int i = 0; i < kFoldMaxPieces; ++i) wts[i] = 0.f;   // no key in any piece: o = 0
                     lse_val = -INFINITY;
                 } else {
-                    const float w_own = fast_exp2(own2 - mx), w_oth = fast_exp2(oth2 - mx);
-                    const float tot = w_own + w_oth;
-                    inv = l_run > 0.f ? dk * w_own / (tot * l_run) : 0.f;
-                    other_w = w_oth / tot;
-                    lse_val = (mx + __log2f(tot)) * 0.69314718055994531f;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kFoldMaxPieces; ++i)
+                        if (i < pieces) sum += expf(wts[i] - m);
+                    lse_val = m + logf(sum);
+#pragma unroll
+                    for (int i = 0; i < kFoldMaxPieces; ++i) wts[i] = i < pieces ? expf(wts[i] - lse_val) : 0.f;
                 }
-                if (!mbar_wait_bounded(bar(kBarFold), 0u, actl)) break;   // one fold per CTA at most
+                if (!mbar_wait_bounded(bar(kBarFold), 0u, actl)) break;
             }
             const bool write_final = direct || fold;
+            bool ep_ok = true;
             // Each warp holds 32 rows.  A step reads 64 tensor-memory columns of its rows (one
             // wait) and moves them, 128 bytes of each row at a time (64 bf16 outputs, or 32 fp32
             // partial columns: two passes), through a per-warp staging area, so that every global
@@ -1035,6 +1158,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 const int row0 = mtile * kRows + kCtaRows * (int)rank + 32 * ((warp - kSoftmaxWarp0) & 1);
 #pragma unroll 1
                 for (int st = 0; st < 4; ++st) {
+                    if (fold && pieces > 2 && st == 2) {
+                        // second fold-in round: columns [256, 512) of the other pieces, once every
+                        // thread has read the first round
+                        mbar_arrive(bar(kBarFoldRd));
+                        if (!mbar_wait_bounded(bar(kBarFoldRd), 0u, actl)) {
+                            ep_ok = false;
+                            break;
+                        }
+                        if (t == 0) fold_issue(1);
+                        if (!mbar_wait_bounded(bar(kBarFold), 1u, actl)) {
+                            ep_ok = false;
+                            break;
+                        }
+                    }
                     uint32_t raw[64];
                     tmem_ld16(tmem + lane_off + kTmemO + 64u * st, *reinterpret_cast<uint32_t(*)[16]>(raw));
                     tmem_ld16(tmem + lane_off + kTmemO + 64u * st + 16u, *reinterpret_cast<uint32_t(*)[16]>(raw + 16));
@@ -1051,20 +1188,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         uint32_t w[32];
                         int col;
                         if (fold) {
-                            // own O (normalised and weighted) + the other piece's row, weighted
+                            // sum over the pieces in slot order of weight x normalised partial row,
+                            // this piece's own from tensor memory (rounded as its stored partial
+                            // would be), the others' from the staged boxes: columns col .. col + 63
+                            // are boxes cb0 and cb0 + 1 of each other piece
                             col = 256 * (st >> 1) + 128 * half + 64 * (st & 1);
-                            // columns col .. col + 63: boxes col / 32 and the next, 16-byte units
-                            // k / 2 = 8 (box) + u at u ^ (rloc & 7) in row rloc of its box
-                            const uint32_t orow = sbase + kOffK + (uint32_t)((col / kFoldBoxCols) * kFoldBoxBytes + rloc * 128);
-#pragma unroll
-                            for (int k = 0; k < 32; k += 2) {
-                                const uint32_t f4 = (uint32_t)(k >> 1);   // float4 index 0 .. 15
-                                const uint4 v = ld_shared_v4u(orow + (f4 >> 3) * (uint32_t)kFoldBoxBytes +
-                                                              (((f4 & 7u) ^ (uint32_t)(rloc & 7)) << 4));
-                                w[k] = pack_bf16x2(__uint_as_float(raw[2 * k]) * inv + __uint_as_float(v.x) * other_w,
-                                                   __uint_as_float(raw[2 * k + 1]) * inv + __uint_as_float(v.y) * other_w);
-                                w[k + 1] = pack_bf16x2(__uint_as_float(raw[2 * k + 2]) * inv + __uint_as_float(v.z) * other_w,
-                                                       __uint_as_float(raw[2 * k + 3]) * inv + __uint_as_float(v.w) * other_w);
+                            const int cb0 = col / kFoldBoxCols;
+                            const uint32_t stg = sbase + kOffQ;
+                            const uint32_t b2 = stg + (uint32_t)cb0 * kFoldBoxBytes;
+                            const uint32_t b30 = stg + (uint32_t)(cb0 & 7) * kFoldBoxBytes;
+                            const uint32_t b31 = stg + (uint32_t)(8 + (cb0 & 7)) * kFoldBoxBytes;
+                            switch (3 * (pieces - 2) + own) {   // uniform over the CTA
+                            case 0: fold_step<2, 0>(raw, w, inv, wts, b2, 0u, rloc); break;
+                            case 1: fold_step<2, 1>(raw, w, inv, wts, b2, 0u, rloc); break;
+                            case 3: fold_step<3, 0>(raw, w, inv, wts, b30, b31, rloc); break;
+                            case 4: fold_step<3, 1>(raw, w, inv, wts, b30, b31, rloc); break;
+                            default: fold_step<3, 2>(raw, w, inv, wts, b30, b31, rloc); break;
                             }
                         } else if (direct) {
 #pragma unroll
@@ -1099,35 +1238,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     }
                 }
             }
+            if (!ep_ok) break;
             if (row_valid && half == 0) {
                 if (write_final)
                     p.lse[(int64_t)ub * p.rows + rowg] = lse_val;
                 else
                     st_global_f32_hint(p.part_lse + (int64_t)split * p.rows + rowg, lse_val, part_pol);
             }
-            if (fold) {
-                // the arrival word is reset for the next call (the other piece counted itself,
-                // this one never does)
-                if (t == 0) *arrival = 0;
-            } else if (!direct && pieces <= kFusedMergeMaxPieces) {
+            if (mode == 1 || mode == 3) {
                 // This piece's partial rows are written: make them visible device-wide, then
-                // count the arrival.  The CTA whose arrival completes the count merges them.
-                // (An mbarrier, not bar.sync, gathers the 128 threads: a bounded wait can never
-                // strand them if another role gave up.)
+                // count them stored (high half of the word); the last claimer merges once all the
+                // others have.  (An mbarrier, not bar.sync, gathers the 128 threads: a bounded
+                // wait can never strand them if another role gave up.)
                 __threadfence();
                 mbar_arrive(bar(kBarPartial));
                 if (!mbar_wait_bounded(bar(kBarPartial), npartial & 1u, actl)) break;
                 ++npartial;
                 if (t == 0) {
-                    int32_t* word = p.arrivals + ((int64_t)ub * gridDim.y + mtile) * 2 + rank;
-                    const int old = atomicAdd(word, 1);
-                    if (old < 0 || old >= pieces) raise_error(128 /* MLA_DEVERR_WORKSPACE_STATE */);
-                    if (old == pieces - 1) {
-                        *word = 0;   // every piece has arrived: ready for the next call
+                    if (mode == 1) {
+                        atomicAdd(arrival, 1 << 16);
+                    } else {
                         const int k = pending[0];
                         if (k < kMaxPendingMerges) {
                             pending[1 + 3 * k] = ub;
-                            pending[2 + 3 * k] = p.num_splits[ub];
+                            pending[2 + 3 * k] = s0;
                             pending[3 + 3 * k] = pieces;
                             pending[0] = k + 1;
                         } else {
@@ -1152,8 +1286,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         const int nrows = min(kCtaRows, p.rows - row_base);
         uint32_t phase = 0;
         auto wait = [&](uint32_t b, uint32_t parity) { return mbar_wait_bounded(b, parity, actl); };
-        for (int k = 0; k < npending && nrows > 0; ++k) {
+        for (int k = 0; k < npending; ++k) {
             const int mb = pending[1 + 3 * k], s0 = pending[2 + 3 * k], n = pending[3 + 3 * k];
+            if (threadIdx.x == 0) {
+                // the other pieces claimed before this one: wait until they have stored
+                int32_t* const word = p.arrivals + ((int64_t)mb * gridDim.y + mtile) * 2 + rank;
+                const bool ok = wait_stored(word, n - 1, actl);
+                if (ok) *word = 0;   // every piece is done with the word: ready for the next call
+                pending[kMiscFold] = ok ? 1 : 0;
+            }
+            __syncthreads();
+            const bool stored_all = pending[kMiscFold] != 0;
+            __syncthreads();   // read before thread 0 can write the flag again
+            if (!stored_all) break;
+            if (nrows <= 0) continue;   // a CTA past the query rows: nothing to write
+            __threadfence();
             if (!merge_rows_cta_bulk<kThreads>(p.part_o, p.part_lse, s0, n, p.rows, row_base, nrows,
                                                p.out + ((int64_t)mb * p.rows + row_base) * kDv,
                                                p.lse + (int64_t)mb * p.rows + row_base,

@@ -82,9 +82,11 @@ mla_status_t prepare_decode_kernels() {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Test hooks (mla_set_test_hooks): the wait budget and the withheld tile of later launches.
+// Test hooks (mla_set_test_hooks): the wait budget, the withheld tile and the fold-in switch of
+// later launches.
 std::atomic<uint64_t> g_hook_wait_budget_ns{0};
 std::atomic<int32_t> g_hook_withhold_tile{-1};
+std::atomic<int32_t> g_hook_no_fold_in{0};
 
 // Workspace layout: arrival words int32 [bs, query tiles, 2], then the split partials
 // fp32 [splits, rows, 512] and their lse fp32 [splits, rows], each 256-byte aligned.
@@ -351,20 +353,31 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     p.part_o = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q));
     p.part_lse = reinterpret_cast<float*>(ws + arrival_bytes(bs, q_len, h_q) +
                                           align256(splits * rows * 512 * sizeof(float)));
-    // part_o as a 2-D fp32 tensor (512 columns [2048 B], splits * rows rows) for the fold-in
-    // merge's loads: boxes of 32 columns x 64 rows, 128-byte swizzle
-    CUtensorMap po_map;
+    // For the fold-in merge's loads: part_o viewed as fp32 [column group (16, 128 B apart)][row
+    // (splits * rows, 2048 B apart)][32 columns], boxes of 8 groups x 64 rows x 32 columns (64 KB,
+    // landing as eight 64-row x 128-byte blocks, 128-byte swizzle); part_lse as [splits][rows],
+    // boxes of 64 rows of one piece (rows a multiple of 4, so that its stride is a multiple of 16
+    // bytes; otherwise no fold-in).
+    CUtensorMap po_map, pl_map;
     std::memset(&po_map, 0, sizeof po_map);
+    std::memset(&pl_map, 0, sizeof pl_map);
     p.fold_ok = 0;
-    if ((uint64_t)splits * (uint64_t)rows <= (uint64_t)INT32_MAX) {
-        const cuuint64_t gdim[2] = {512, (cuuint64_t)splits * (cuuint64_t)rows};
-        const cuuint64_t gstride[1] = {512 * sizeof(float)};
-        const cuuint32_t box[2] = {(cuuint32_t)mla::decode::kFoldBoxCols, (cuuint32_t)mla::decode::kCtaRows};
-        const cuuint32_t estride[2] = {1, 1};
-        if (encode(&po_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.part_o, gdim, gstride, box, estride,
+    if ((uint64_t)splits * (uint64_t)rows <= (uint64_t)INT32_MAX && rows % 4 == 0) {
+        const cuuint64_t gdim[3] = {(cuuint64_t)mla::decode::kFoldBoxCols, (cuuint64_t)splits * (cuuint64_t)rows,
+                                    512 / (cuuint64_t)mla::decode::kFoldBoxCols};
+        const cuuint64_t gstride[2] = {512 * sizeof(float), mla::decode::kFoldBoxCols * sizeof(float)};
+        const cuuint32_t box[3] = {(cuuint32_t)mla::decode::kFoldBoxCols, (cuuint32_t)mla::decode::kCtaRows, 8};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        const cuuint64_t ldim[2] = {(cuuint64_t)rows, (cuuint64_t)splits};
+        const cuuint64_t lstride[1] = {(cuuint64_t)rows * sizeof(float)};
+        const cuuint32_t lbox[2] = {(cuuint32_t)mla::decode::kCtaRows, 1};
+        if (encode(&po_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.part_o, gdim, gstride, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+            encode(&pl_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.part_lse, ldim, lstride, lbox, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-            p.fold_ok = 1;
+            p.fold_ok = g_hook_no_fold_in.load(std::memory_order_relaxed) ? 0 : 1;
     }
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -372,13 +385,13 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     using mla::decode::kSmemBytes;
     using mla::decode::kThreads;
     if (q_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
+        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
+        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E5M2)
-        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
+        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
     else
-        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, p);
+        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
@@ -545,10 +558,11 @@ mla_status_t mla_extend_paged_prefix(const void* q, int32_t bs, int32_t e, int32
                            reinterpret_cast<const float*>(at(L.lse2)), (int64_t)rows, 512, out, lse, stream);
 }
 
-mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile) {
+mla_status_t mla_set_test_hooks(uint64_t wait_budget_ns, int32_t withhold_tile, int32_t no_fold_in) {
     if (withhold_tile < -1) return MLA_ERR_INVALID_ARG;
     g_hook_wait_budget_ns.store(wait_budget_ns, std::memory_order_relaxed);
     g_hook_withhold_tile.store(withhold_tile, std::memory_order_relaxed);
+    g_hook_no_fold_in.store(no_fold_in != 0, std::memory_order_relaxed);
     return MLA_OK;
 }
 

@@ -96,8 +96,8 @@ def test_decode_validation_happens_before_any_launch():
 
 def test_test_hooks_validation():
     lib = mla.library()
-    assert lib.mla_set_test_hooks(0, -2) == 1
-    assert lib.mla_set_test_hooks(0, -1) == 0     # the defaults (no launch involved)
+    assert lib.mla_set_test_hooks(0, -2, 0) == 1
+    assert lib.mla_set_test_hooks(0, -1, 0) == 0     # the defaults (no launch involved)
 
 
 def test_set_kv_buffer_validation():

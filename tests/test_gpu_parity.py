@@ -537,6 +537,53 @@ def test_repeated_calls_on_one_workspace_are_identical(mla):
     assert mla.read_device_error() == 0
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", ["decode", "verify", "fp8"])
+def test_fold_in_and_stored_merge_agree_bit_for_bit(mla, case):
+    """The last piece of a split request either folds the other pieces' partial rows into its own
+    result or stores its partial and merges the stored ones at the end of its part; both sum the
+    pieces in split-slot order with the same weights, so the results agree bit for bit (and
+    whichever piece happens to finish last, the output is the same).  Nine forced parts give
+    requests of two and three pieces (four in the verify case)."""
+    if case == "decode":
+        wl = W.make_case([700, 1500, 64, 2300, 1, 900], 128, seed=81)
+    elif case == "verify":
+        wl = W.make_case([700, 1500, 64, 2300, 3], 64, q_len=4, verify=True, seed=82)
+    else:
+        wl = W.make_case([700, 1500, 64, 2300, 1, 900], 128, kv="fp8", seed=83)
+    g = wl.to("cuda")
+    bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages,
+                               seq_len_add=wl.num_draft_tokens)
+    parts = 9
+    md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, 1, wl.is_fp8, num_parts=parts)
+    pieces = np.diff(ns.cpu().numpy())
+    assert ({3, 4} if case == "verify" else {2, 3}) <= set(pieces.tolist()), pieces
+    ws = torch.zeros((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), dtype=torch.uint8, device="cuda")
+    tiles = -(-(wl.q_len * wl.h) // 128)
+    arrival = -(-wl.bs * tiles * 2 * 4 // 256) * 256
+    outs = []
+    try:
+        for no_fold in (False, True, False):
+            mla.set_test_hooks(0, -1, no_fold_in=no_fold)
+            o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                                          wl.causal, g.descale_q, g.descale_k, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.count_nonzero(ws[:arrival]) == 0, "every call leaves the arrival words zero"
+            outs.append((o.clone(), lse.clone()))
+    finally:
+        mla.set_test_hooks(0, -1, no_fold_in=False)
+    assert mla.read_device_error() == 0
+    for o, lse in outs[1:]:
+        assert torch.equal(o, outs[0][0]), "fold-in and stored merge differ"
+        assert torch.equal(lse, outs[0][1]), "fold-in and stored merge differ (lse)"
+    ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
+                                       wl.cache_seqlens, wl.softmax_scale, wl.causal, kv_is_fp8=wl.is_fp8,
+                                       descale_q=float(wl.descale_q[0]) if wl.descale_q is not None else 1.0,
+                                       descale_k=float(wl.descale_k[0]) if wl.descale_k is not None else 1.0)
+    o, lse = outs[0]
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "fold-in " + case)
+
+
 def test_unzeroed_workspace_is_reported(mla):
     """A workspace whose arrival words are not zero (never zero-filled) is reported in the
     error word; zero-filling it makes the next call correct again."""
