@@ -160,8 +160,10 @@ __device__ __forceinline__ bool merge_rows_cta_bulk(const float* __restrict__ pa
 // The rows of requests of more than kFusedMergeMaxPieces pieces (the others were written whole or
 // merged by the attention kernel, so the launch needs no host knowledge of the plan): each CTA
 // first stages num_splits in shared memory (one coalesced read, for up to kCombineStagedRequests
-// requests), then its warps take (request, query row) pairs in turn; a grid of about one CTA per
-// SM, so that a batch with nothing left to merge costs one pass over the plan.
+// requests) and notes whether any request has that many pieces, then waits for the attention
+// grid; its warps then take (request, query row) pairs in turn, or the CTA returns at once when
+// nothing is left to merge.  num_splits comes from the metadata step, which completed before the
+// attention kernel started, so it is read while the attention kernel still runs.
 constexpr int kCombineStagedRequests = 4096;
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
@@ -169,13 +171,21 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
                       const int32_t* __restrict__ num_splits, int32_t rows, int32_t bs,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
     __shared__ int32_t s_ns[kCombineStagedRequests + 1];
-    // launched as a programmatic dependent of the attention kernel: wait for all of it
-    pdl_wait_prerequisites();
     const bool staged = bs <= kCombineStagedRequests;
+    int many = 0;   // some request of this thread's has more pieces than the attention kernel merges
     if (staged) {
         for (int b = threadIdx.x; b <= bs; b += blockDim.x) s_ns[b] = num_splits[b];
         __syncthreads();
+        for (int b = threadIdx.x; b < bs; b += blockDim.x) many |= s_ns[b + 1] - s_ns[b] > kFusedMergeMaxPieces;
+    } else {
+        for (int b = threadIdx.x; b < bs; b += blockDim.x)
+            many |= num_splits[b + 1] - num_splits[b] > kFusedMergeMaxPieces;
     }
+    many = __syncthreads_or(many);
+    // launched as a programmatic dependent of the attention kernel: wait for all of it (also when
+    // there is nothing to merge, so that this grid never completes before the one it follows)
+    pdl_wait_prerequisites();
+    if (!many) return;
     const uint64_t read_pol = l2_policy_evict_first();   // the partials are read once
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * kCombineWarps;
