@@ -98,7 +98,7 @@ TRAFFIC_KEYS = {2: "deepseek_v3_decode"}
 
 # The sources the decode kernel is built from: its body, the PTX helpers it inlines, and the
 # translation unit with its tensor maps and launch configuration.
-DECODE_KERNEL_SOURCES = ("decode.cuh", "ptx.cuh", "mla_b200.cu")
+DECODE_KERNEL_SOURCES = ("decode.cuh", "combine.cuh", "ptx.cuh", "mla_b200.cu")
 
 
 def kernel_sources_sha():
