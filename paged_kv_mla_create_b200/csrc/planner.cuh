@@ -132,6 +132,7 @@ __device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t par
         // off the common path.
         int i = 0, r = P, cum = 0;
         int nb = s_nb[0];
+#pragma unroll 4
         for (int b = 0; b < bs; ++b) {
             const int nb_next = s_nb[b + 1];
             const int c = nb + kFixedOverhead;
