@@ -188,8 +188,9 @@ MLA_API mla_status_t mla_build_decode_metadata(
 
 /*
  * Bytes of workspace mla_decode_paged needs, 256-byte aligned parts in this order:
- *   arrival words  int32 [bs, cdiv(q_len * h_q, 128), 2]: split pieces of a request count
- *                  their arrival here, and the last to arrive merges the request's rows
+ *   arrival words  int32 [bs, cdiv(q_len * h_q, 128), 2]: split pieces of a request claim a
+ *                  place and count their stored partials here, and the last to claim merges
+ *                  the request's rows
  *                  (requests of up to 4 pieces); every completed call leaves them zero;
  *   partial outputs fp32 [(bs + num_sm_parts) * q_len * h_q, 512] and their log-sum-exps.
  * Pure host function; returns 0 on a non-positive argument.
