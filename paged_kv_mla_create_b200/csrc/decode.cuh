@@ -95,7 +95,8 @@ constexpr int kOffQ = 0;                            // Q chunks 4..8
 constexpr int kOffK = kOffQ + kQHiBytes;
 constexpr int kOffP = kOffK + kKSlots * kKSlotBytes;
 constexpr int kOffX = kOffP + kPBytes;              // row-max exchange: 2 x 128 floats, row sums 128
-constexpr int kOffStage = kOffX + 3 * 128 * 4;      // epilogue staging: 4 warps x 32 rows x 128 B
+constexpr int kOffStage = kOffX + 3 * 1024;         // epilogue staging: 4 warps x 32 rows x 128 B
+                                                    // (1 KB aligned: boxes of TMA stores, 128-byte swizzle)
 constexpr int kOffPSig = kOffStage + 4 * 32 * 128;  // leader: landing words of the peer's P signals
 constexpr int kOffBar = kOffPSig + 128;   // landing words: P 0..3, V 4..7, K 8, Q 9..12,
                                             // S read 16..19, O read 20..23
@@ -153,7 +154,9 @@ static_assert(kFoldBoxes * kFoldBoxBytes <= kOffX - kOffQ &&
 constexpr int kMaxPendingMerges = 2;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
+static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0 && kOffStage % 1024 == 0,
+              "128-byte swizzle atoms need 1 KB alignment");
+static_assert(kOffStage >= kOffX + 3 * 128 * 4, "the exchange area fits before the staging");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
@@ -390,7 +393,8 @@ template <int kKv, bool kFp8Q>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
                   const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap po_map,
-                  const __grid_constant__ CUtensorMap pl_map, const __grid_constant__ Params p) {
+                  const __grid_constant__ CUtensorMap pl_map, const __grid_constant__ CUtensorMap o_map,
+                  const __grid_constant__ CUtensorMap ps_map, const __grid_constant__ Params p) {
     constexpr bool kFp8 = kKv != 0;
     constexpr bool kE5M2 = kKv == 2;
     static_assert(kKv == 1 || !kFp8Q, "e4m3 queries need an e4m3 cache");
@@ -468,6 +472,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         prefetch_tensormap(&q_map);
         prefetch_tensormap(&po_map);
         prefetch_tensormap(&pl_map);
+        prefetch_tensormap(&o_map);
+        prefetch_tensormap(&ps_map);
     }
     tc_fence_before();
     __syncthreads();
@@ -1154,7 +1160,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             // store writes whole 128-byte lines (8 lanes per row).  TMEM columns [128 + 64 st, +64)
             // hold outputs 256 (st / 2) + 128 half + 64 (st % 2) + [0, 64).
             {
-                const uint32_t stage = sbase + kOffStage + (uint32_t)(warp - kSoftmaxWarp0) * 4096u;
+                // staging: the warp's own 4 KB and its 4 KB of the P buffer (idle until this
+                // warp writes the next unit's first P)
+                const uint32_t stage_a = sbase + kOffStage + (uint32_t)(warp - kSoftmaxWarp0) * 4096u;
+                const uint32_t stage_b = sbase + kOffP + (uint32_t)(warp - kSoftmaxWarp0) * 4096u;
+                uint32_t npass = 0;
                 const int row0 = mtile * kRows + kCtaRows * (int)rank + 32 * ((warp - kSoftmaxWarp0) & 1);
 #pragma unroll 1
                 for (int st = 0; st < 4; ++st) {
@@ -1215,29 +1225,42 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                             for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(raw[32 * pass + k]) * inv);
                             col = 256 * (st >> 1) + 128 * half + 64 * (st & 1) + 32 * pass;
                         }
-                        // this thread's 128 bytes -> staging row `lane` (16-byte unit k at k ^ (lane & 7))
+                        // this thread's 128 bytes -> staging row `lane` (16-byte unit k at k ^ (lane & 7), the
+                        // 128-byte swizzle of a 32-row x 128-byte box), then one TMA store of the box
+                        // (rows past the request's last are clipped).  Two staging buffers alternate;
+                        // a buffer is rewritten once the store that used it has read it.
+                        const uint32_t stage = (npass & 1u) ? stage_b : stage_a;
+                        if (lane == 0 && npass >= 2) bulk_wait_read<1>();
+                        __syncwarp();
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             st_shared_v4u(stage + (uint32_t)lane * 128u + 16u * ((uint32_t)k ^ ((uint32_t)lane & 7u)),
                                           w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        fence_proxy_async_smem();
                         __syncwarp();
-                        // 4 rows per store instruction, 8 lanes (128 contiguous bytes) per row
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int r = 4 * j + (lane >> 3), u = lane & 7;
-                            const int rg = row0 + r;
-                            const uint4 v = ld_shared_v4u(stage + (uint32_t)r * 128u + 16u * ((uint32_t)u ^ ((uint32_t)r & 7u)));
-                            if (rg < p.rows) {
-                                if (write_final)
-                                    *reinterpret_cast<uint4*>(p.out + ((int64_t)ub * p.rows + rg) * kDv + col + 8 * u) = v;
-                                else
-                                    st_global_v4_hint(p.part_o + ((int64_t)split * p.rows + rg) * kDv + col + 4 * u, v, part_pol);
-                            }
+                        if (lane == 0 && row0 < p.rows) {   // (a warp past the request's rows stores nothing)
+                            if (write_final)
+                                tma_store_3d(&o_map, stage, col, row0, ub);
+                            else
+                                tma_store_3d_hint(&ps_map, stage, col, row0, split, part_pol);
+                            bulk_commit();
                         }
+                        ++npass;
                         __syncwarp();
                     }
                 }
             }
+            // the staging (and the P buffer) free again; a stored piece's rows also complete (their
+            // count below makes them visible to other CTAs, whose loads go through the async proxy)
+            if (lane == 0) {
+                if (write_final) {
+                    bulk_wait_read<0>();
+                } else {
+                    bulk_wait<0>();
+                    fence_proxy_async_global();
+                }
+            }
+            __syncwarp();
             if (!ep_ok) break;
             if (row_valid && half == 0) {
                 if (write_final)
@@ -1274,6 +1297,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         }
     }
 
+    if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + 4 && lane == 0) bulk_wait<0>();   // the epilogues' stores
     tc_fence_before();
     __syncthreads();
     // Merges of the requests whose last piece arrived here, by the whole CTA: the pieces' rows

@@ -379,19 +379,41 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
             p.fold_ok = g_hook_no_fold_in.load(std::memory_order_relaxed) ? 0 : 1;
     }
+    // The epilogue's stores: o bf16 viewed as [bs][rows][512] in boxes of 32 rows x 64 columns, the
+    // partials fp32 [splits][rows][512] in boxes of 32 rows x 32 columns (128 bytes a row, 128-byte
+    // swizzle); rows past a request's last are clipped by the view.
+    CUtensorMap o_map, ps_map;
+    std::memset(&o_map, 0, sizeof o_map);
+    std::memset(&ps_map, 0, sizeof ps_map);
+    {
+        const cuuint64_t odim[3] = {512, (cuuint64_t)rows, (cuuint64_t)bs};
+        const cuuint64_t ostride[2] = {512 * 2, (cuuint64_t)rows * 512 * 2};
+        const cuuint32_t obox[3] = {64, 32, 1};
+        const cuuint64_t sdim[3] = {512, (cuuint64_t)rows, (cuuint64_t)splits};
+        const cuuint64_t sstride[2] = {512 * 4, (cuuint64_t)rows * 512 * 4};
+        const cuuint32_t sbox[3] = {32, 32, 1};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        if (encode(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, odim, ostride, obox, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+            encode(&ps_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.part_o, sdim, sstride, sbox, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
     using mla::decode::kSmemBytes;
     using mla::decode::kThreads;
     if (q_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
+        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
+        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E5M2)
-        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
+        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else
-        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, p);
+        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
