@@ -32,13 +32,14 @@
 //     load Q once per unit (columns [256, 576) by TMA into shared memory, columns [0, 256)
 //     into tensor memory), and warp 11 loads the partner V of every tile by TMA once the
 //     tile's S is done (an e4m3 cache: all four warps, through registers, widening to f16),
-//     and prefetch the later units' query rows into L2; warp 1 lane 0 of the leader issues
-//     every MMA; warps 4..7 (thread t = TMEM lane t: row t % 64, token half
+//     and prefetch the later units' query rows into L2; warp 1 of the leader walks the MMA
+//     schedule and an elected lane issues every MMA; warps 4..7 (thread t = TMEM lane t: row t % 64, token half
 //     t / 64) run the online softmax: partner threads t and t ^ 64 agree on each row's
 //     maximum through shared memory (an mbarrier orders the exchange, so a timed-out wait
 //     can never strand the others), P goes to shared memory for the PV MMA, O is rescaled
 //     in tensor memory only when the running maximum grows by more than 2^8, and the
-//     epilogue normalises and writes o and lse.
+//     epilogue normalises o (or keeps fp32 partials) and writes it as TMA stores of
+//     32-row boxes staged in shared memory, and writes lse.
 //   * A unit whose block range is a whole request writes bf16 o and lse directly.  A piece of a
 //     request of at most kFusedMergeMaxPieces pieces claims a place on a per-(request, query
 //     tile, CTA) word of the workspace during its last tile; the last to claim merges the
