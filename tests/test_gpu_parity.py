@@ -584,6 +584,43 @@ def test_fold_in_and_stored_merge_agree_bit_for_bit(mla, case):
     assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "fold-in " + case)
 
 
+def test_random_split_batches(mla):
+    """Random batches over forced part counts, so that requests split into one to many pieces in
+    every arrangement the planner makes: each case against the oracle, then run again on the same
+    workspace, which must give the same bits (whichever piece of a request happens to merge) and
+    leave the arrival words zero."""
+    rng = np.random.default_rng(2026)
+    for case in range(24):
+        h = int(rng.choice([16, 64, 128]))
+        q_len = int(rng.choice([1, 1, 2]))
+        bs = int(rng.integers(1, 7))
+        lens = [int(x) for x in rng.choice([0, 1, 63, 64, 65, 200, 700, 1500, 2300], size=bs)]
+        if max(lens) == 0:
+            lens[0] = 129
+        parts = int(rng.integers(2, 20))
+        wl = W.make_case(lens, h, q_len=q_len, verify=q_len > 1, seed=3000 + case)
+        g = wl.to("cuda")
+        bt = mla.build_block_table(g.req_to_token, g.req_pool_indices, g.seq_lens, wl.max_pages,
+                                   seq_len_add=wl.num_draft_tokens)
+        md, ns = mla.get_mla_metadata(g.cache_seqlens, wl.q_len * wl.h, 1, False, num_parts=parts)
+        ws = torch.zeros((mla.workspace_bytes(wl.bs, wl.q_len, wl.h, parts),), dtype=torch.uint8, device="cuda")
+        tiles = -(-(wl.q_len * wl.h) // 128)
+        arrival = -(-wl.bs * tiles * 2 * 4 // 256) * 256
+        outs = []
+        for _ in range(2):
+            o, lse = mla.mla_decode_paged(g.q, g.kv_cache, bt, g.cache_seqlens, 512, md, ns, wl.softmax_scale,
+                                          wl.causal, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.count_nonzero(ws[:arrival]) == 0, f"case {case}: arrival words left set"
+            outs.append((o.clone(), lse.clone()))
+        assert mla.read_device_error() == 0, f"case {case}"
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1]), f"case {case}: bits differ"
+        ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, wl.req_pool_indices,
+                                           wl.cache_seqlens, wl.softmax_scale, wl.causal)
+        assert_close(outs[0][0].float().cpu().numpy(), outs[0][1].cpu().numpy(), ref_o, ref_lse,
+                     f"random case {case} (lens {lens}, h {h}, q_len {q_len}, parts {parts})")
+
+
 def test_unzeroed_workspace_is_reported(mla):
     """A workspace whose arrival words are not zero (never zero-filled) is reported in the
     error word; zero-filling it makes the next call correct again."""
