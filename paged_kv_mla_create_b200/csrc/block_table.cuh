@@ -57,6 +57,7 @@ build_block_table_kernel(const int32_t* __restrict__ req_to_token, int64_t r2t_r
                          const LenT* __restrict__ seq_lens, int32_t seq_len_add,
                          int32_t* __restrict__ block_table, int64_t bt_stride,
                          int32_t max_pages, int32_t fill_tail) {
+    pdl_launch_dependents();   // a programmatic dependent waits for this grid's completion
     const int b = blockIdx.x;
     const int p = blockIdx.y * blockDim.x + threadIdx.x;
     if (p >= max_pages) return;
@@ -75,6 +76,9 @@ decode_metadata_kernel(const int32_t* __restrict__ req_to_token, int64_t r2t_row
                        int64_t bt_stride, int32_t max_pages, int32_t fill_tail, int32_t parts,
                        int32_t* __restrict__ cache_seqlens, int32_t* __restrict__ md,
                        int32_t* __restrict__ num_splits) {
+    // The attention grid, launched as a programmatic dependent, may be scheduled now: it sets
+    // itself up and then waits for this grid to complete before it reads any of its outputs.
+    pdl_launch_dependents();
     if (blockIdx.x == 0) {
         __shared__ PlannerSmem sm;
         plan_parts(

@@ -162,8 +162,9 @@ __device__ __forceinline__ bool merge_rows_cta_bulk(const float* __restrict__ pa
 // first stages num_splits in shared memory (one coalesced read, for up to kCombineStagedRequests
 // requests) and notes whether any request has that many pieces, then waits for the attention
 // grid; its warps then take (request, query row) pairs in turn, or the CTA returns at once when
-// nothing is left to merge.  num_splits comes from the metadata step, which completed before the
-// attention kernel started, so it is read while the attention kernel still runs.
+// nothing is left to merge.  num_splits comes from the metadata step: the attention kernel lets
+// this grid in only after its own wait for that step to complete, so num_splits is final and is
+// read while the attention kernel still runs.
 constexpr int kCombineStagedRequests = 4096;
 
 __global__ void __launch_bounds__(kCombineWarps * 32)

@@ -414,19 +414,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const bool leader = rank == 0;
     const int part = blockIdx.x >> 1;
     const int mtile = blockIdx.y;
-    // The merge kernel that follows waits for this whole grid anyway; let it be scheduled
-    // now, so that its launch overlaps this kernel.
-    pdl_launch_dependents();
-    // The part's plan row first, and the first request's length and page ids it points at
-    // fetched into L2, so that their latency overlaps the set-up below rather than delaying the
-    // first page load.
-    bool md_ok = true;
-    UnitIter iter = make_iter(p, part, md_ok);
-    if (warp == 0 && md_ok && iter.b < p.bs) {
-        if (lane == 0) prefetch_l2(p.cache_seqlens + iter.b);
-        const int blk = iter.k0 + lane;
-        if (blk < p.max_pages) prefetch_l2(p.block_table + (int64_t)iter.b * p.bt_stride + blk);
-    }
+    // Launched as a programmatic dependent of the metadata step, this grid is scheduled while
+    // that step still runs: the set-up below (barriers, tensor memory, descriptors) reads
+    // nothing another grid writes, and overlaps it.
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKSlots; ++s) {
@@ -480,6 +470,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     __syncthreads();
     cluster_sync();
     tc_fence_after();
+    // Everything from here on may read what the preceding grids wrote (plan, page table,
+    // lengths, queries, cache, the workspace's arrival words): wait for them to complete.
+    // Without a programmatic launch this returns at once.  Only then is the merge kernel that
+    // follows let in, since it reads num_splits before it waits for this grid.
+    pdl_wait_prerequisites();
+    pdl_launch_dependents();
+    bool md_ok = true;
+    UnitIter iter = make_iter(p, part, md_ok);
     const uint32_t tmem = *tmem_slot;
     // (the partner's flag was zeroed before the cluster barrier above)
     const AbortCtl actl{abort_flag, map_to_cta(smem_u32(tmem_slot + 1), rank ^ 1u), p.wait_budget_ns};

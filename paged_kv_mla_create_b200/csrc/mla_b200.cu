@@ -406,15 +406,29 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     const dim3 grid(2 * num_sm_parts, (rows + 127) / 128);
     using mla::decode::kSmemBytes;
     using mla::decode::kThreads;
+    // A programmatic dependent launch (the pair size comes from the kernel's cluster
+    // dimensions): when the grid before it in the stream lets it in early, as the metadata
+    // kernels do, its set-up overlaps that grid; it waits for that grid to complete before it
+    // reads anything (with any other predecessor it starts once that one has completed).
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t dcfg = {};
+    dcfg.gridDim = grid;
+    dcfg.blockDim = dim3(kThreads);
+    dcfg.dynamicSmemBytes = kSmemBytes;
+    dcfg.stream = s;
+    dcfg.attrs = pdl;
+    dcfg.numAttrs = 1;
+    cudaError_t e;
     if (q_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, true><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
+        e = cudaLaunchKernelEx(&dcfg, mla::decode::mla_decode_kernel<1, true>, k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E4M3)
-        mla::decode::mla_decode_kernel<1, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
+        e = cudaLaunchKernelEx(&dcfg, mla::decode::mla_decode_kernel<1, false>, k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else if (kv_dtype == MLA_DTYPE_FP8_E5M2)
-        mla::decode::mla_decode_kernel<2, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
+        e = cudaLaunchKernelEx(&dcfg, mla::decode::mla_decode_kernel<2, false>, k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     else
-        mla::decode::mla_decode_kernel<0, false><<<grid, kThreads, kSmemBytes, s>>>(k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
-    cudaError_t e = cudaGetLastError();
+        e = cudaLaunchKernelEx(&dcfg, mla::decode::mla_decode_kernel<0, false>, k_map, v_map, q_map, po_map, pl_map, o_map, ps_map, p);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     // The merge of requests of many pieces, as a programmatic dependent launch: scheduled while
     // the attention kernel runs, it waits on the device for that grid to complete.
@@ -427,10 +441,7 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     cfg.blockDim = dim3(mla::kCombineWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
+    cfg.attrs = pdl;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, mla::combine_splits_kernel, (const float*)p.part_o, (const float*)p.part_lse,
                            num_splits, rows, bs, p.out, lse);

@@ -205,6 +205,7 @@ __global__ void __launch_bounds__(kPlannerThreads)
 get_mla_metadata_kernel(const int32_t* __restrict__ cache_seqlens, int32_t bs, int32_t parts,
                         int32_t* __restrict__ md, int32_t* __restrict__ num_splits) {
     __shared__ PlannerSmem sm;
+    pdl_launch_dependents();   // a programmatic dependent waits for this grid's completion
     plan_parts([&](int b) -> int32_t { return cache_seqlens[b]; }, bs, parts, md, num_splits, nullptr, sm);
 }
 
