@@ -13,7 +13,7 @@
 // part i's budget left, either it fits (r >= blocks + F), or, after skipping to a fresh
 // part when r <= F, its first piece takes r - F blocks, the following parts take
 // Q = P - F blocks each, and the last piece takes the rest (1..Q blocks) -- a closed form
-// whose one division is needed only when a request spans more than one further part.  One
+// whose one division is needed only when a request spans more than two further parts.  One
 // thread runs that O(bs) recurrence, a short chain of compares per request; then one thread
 // per part reads its row off the per-request results by binary search: its first piece
 // belongs to the first request whose last part is >= i, its last to the last request
@@ -27,18 +27,6 @@ namespace mla {
 constexpr int kFixedOverhead = 5;        // blocks of cost charged per piece
 constexpr int kPlannerThreads = 256;
 constexpr int kPlannerSmemLens = 2048;   // requests handled by the per-request walk
-
-// a / q for 0 <= a < 2^31, q >= 1: a float estimate (q_inv = 1 / q) corrected to the exact
-// quotient, much shorter on the walk's dependency chain than an integer division.
-__device__ __forceinline__ int div_small(int a, int q, float q_inv) {
-    int m = __float2int_rz((float)a * q_inv);
-    // one step each way covers the estimate's error for a < 2^22; the loops finish the rest
-    m = (m > 0 && m * q > a) ? m - 1 : m;
-    m = ((m + 1) * q <= a) ? m + 1 : m;
-    while (m > 0 && m * q > a) --m;
-    while ((m + 1) * q <= a) ++m;
-    return m;
-}
 
 struct PlannerSmem {
     int32_t nb[kPlannerSmemLens + 1];   // blocks of request b
@@ -81,7 +69,6 @@ __device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t par
     // Budgets fit in 32 bits for any table a decode step can address (< 2^31 blocks).
     const int P = (int)((total + parts - 1) / parts) + kFixedOverhead;
     const int Q = P - kFixedOverhead;   // >= 1
-    const float qinv = 1.0f / (float)Q;
 
     if (!staged) {
         // part-by-part walk, lengths from global memory
@@ -128,8 +115,10 @@ __device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t par
         // Entering request b of c = blocks + F: a part with r <= F and r < c ends unused; the
         // request then fits (r >= c) or is split: its first piece takes r - F blocks, m full
         // middle parts take Q blocks each and the last piece the rest, last = rem - m Q with
-        // rem = c - r, leaving Q - last.  m > 0 only when rem - 1 >= Q, so the division stays
-        // off the common path.
+        // rem = c - r, leaving Q - last.  m = (rem - 1) / Q is 0 or 1 unless the request spans
+        // more than two further parts, so the division stays off the common path: a request
+        // about as long as a part's budget often spans two, and a float-estimate quotient or a
+        // modulo on that path cost ~30 cycles a request more (bs 64, budget 44 blocks).
         int i = 0, r = P, cum = 0;
         int nb = s_nb[0];
 #pragma unroll 4
@@ -147,7 +136,8 @@ __device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t par
                 cum += 1;
             } else {
                 const int rem = c - r;                                   // >= 1
-                const int m = rem - 1 >= Q ? div_small(rem - 1, Q, qinv) : 0;
+                int m = rem > Q ? 1 : 0;
+                if (rem > 2 * Q) m = (rem - 1) / Q;
                 s_x0[b] = r - kFixedOverhead;                            // 1 <= x0 < nb
                 i += 1 + m;
                 r = Q - (rem - m * Q);
