@@ -93,7 +93,7 @@ def job_value(world, kv_bytes_per_replica, step_ms):
     return world * kv_bytes_per_replica / (step_ms * 1e-3) / 1e9
 
 
-TRAFFIC_KEYS = {2: "deepseek_v3_decode"}
+TRAFFIC_KEYS = {2: "deepseek_v3_decode", 3: "skewed_long_context", 4: "fp8_kv_decode", 5: "target_verify"}
 
 
 # The sources the decode kernel is built from: its body, the PTX helpers it inlines, and the
@@ -338,6 +338,8 @@ class Case:
         import paged_kv_mla_create_b200 as mla
         from paged_kv_mla_create_b200 import workloads as W
         self.mla, self.dev, self.cfg = mla, dev, cfg
+        # the committed DRAM capture that belongs to this workload's kernel (none for e4m3 q)
+        self.traffic_key = None if q_fp8 else cfg
         self.host = host = W.make_workload(cfg, seed=seed, q_fp8=q_fp8)
         self.wl = host.to(dev)
         self.kv_bytes, self.q_bytes, self.flops = algorithmic(host)
@@ -540,6 +542,7 @@ class ExtendCase(Case):
         import paged_kv_mla_create_b200 as mla
         from paged_kv_mla_create_b200 import workloads as W
         self.mla, self.dev, self.cfg = mla, dev, "extend"
+        self.traffic_key = None
         rng = np.random.default_rng(seed)
         prefix = [int(x) for x in rng.integers(1024, 4097, size=4)]
         e = 64
@@ -591,7 +594,7 @@ def config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src):
             "kv_gbs_per_call": case.kv_bytes / attn_s / 1e9, "tflops": case.flops / attn_s / 1e12,
             "kv_bytes": case.kv_bytes, "q_bytes": case.q_bytes, "flops": case.flops,
             "roofline": roofline_entry(case.kv_bytes, case.q_bytes, case.flops, attn_s, peaks,
-                                       peak_src, case.host.is_fp8, captured_traffic(case.cfg)),
+                                       peak_src, case.host.is_fp8, captured_traffic(case.traffic_key)),
             "clocks": clk}
 
 

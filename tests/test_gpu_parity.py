@@ -726,3 +726,68 @@ def test_extend_with_fp8_prefix(mla):
     assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, "extend, e4m3 prefix",
                  max_abs=EXTEND_MAX_ABS)
     assert mla.read_device_error() == 0
+
+
+# ------------------------------------------------------------------ one CUDA graph per step
+def test_metadata_and_attention_in_one_graph_follow_new_batches(mla):
+    """Metadata and attention captured in one CUDA graph, the way the benchmark replays a step:
+    the attention kernel is a programmatic dependent of the metadata kernel, scheduled while the
+    plan is still being computed.  Between replays the batch changes (new lengths, requests
+    mapped to other rows of req_to_token), so an attention grid that read any of the plan, page
+    table or lengths before the metadata grid had finished would attend the previous batch.
+    Every replay is checked against the oracle for its own batch; the metadata bit for bit."""
+    rng = np.random.default_rng(4242)
+    lens = [3000, 700, 4100, 64, 1500, 2500, 130, 3900]
+    wl = W.make_case(lens, 128, seed=4242)
+    g = wl.to("cuda")
+    alloc = {int(wl.req_pool_indices[b]): lens[b] for b in range(wl.bs)}
+    batches = [(wl.req_pool_indices.clone(), wl.seq_lens.clone())]
+    for _ in range(3):
+        rpi = wl.req_pool_indices[torch.from_numpy(rng.permutation(wl.bs))]
+        sl = torch.tensor([int(rng.integers(1, alloc[int(r)] + 1)) for r in rpi], dtype=torch.int32)
+        batches.append((rpi.clone(), sl))
+    batches.append(batches[0])
+    rpi_d, sl_d = g.req_pool_indices.clone(), g.seq_lens.clone()
+    parts = mla.num_sm_parts(wl.q_len * wl.h)
+    bt = torch.empty((wl.bs, wl.max_pages), dtype=torch.int32, device="cuda")
+    cl = torch.empty((wl.bs,), dtype=torch.int32, device="cuda")
+    md = torch.empty((parts, 8), dtype=torch.int32, device="cuda")
+    ns = torch.empty((wl.bs + 1,), dtype=torch.int32, device="cuda")
+    o = torch.empty((wl.bs, 1, wl.h, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.bs, 1, wl.h), dtype=torch.float32, device="cuda")
+    ws = torch.zeros((mla.workspace_bytes(wl.bs, 1, wl.h, parts),), dtype=torch.uint8, device="cuda")
+
+    def step():
+        mla.build_decode_metadata(g.req_to_token, rpi_d, sl_d, wl.max_pages, wl.h, 1, False,
+                                  out=(bt, cl, md, ns))
+        mla.mla_decode_paged(g.q, g.kv_cache, bt, cl, 512, md, ns, wl.softmax_scale, True,
+                             out=o, lse=lse, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    try:
+        for t, (rpi, sl) in enumerate(batches):
+            rpi_d.copy_(rpi)
+            sl_d.copy_(sl)
+            graph.replay()
+            torch.cuda.synchronize()
+            ref_bt = oracle.build_block_table(wl.req_to_token, rpi, sl, wl.max_pages)
+            ref_md, ref_ns = oracle.get_mla_metadata(sl.numpy(), parts)
+            assert np.array_equal(bt.cpu().numpy(), ref_bt), f"replay {t}: page table"
+            assert np.array_equal(cl.cpu().numpy(), sl.numpy()), f"replay {t}: lengths"
+            assert np.array_equal(md.cpu().numpy(), ref_md), f"replay {t}: plan"
+            assert np.array_equal(ns.cpu().numpy(), ref_ns), f"replay {t}: num_splits"
+            ref_o, ref_lse = oracle.mla_decode(wl.q, wl.kv_cache, wl.req_to_token, rpi, sl,
+                                               wl.softmax_scale, True)
+            assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse, f"replay {t}")
+        assert int(ns[-1]) > 4 * wl.bs, "the batch should split requests into many pieces"
+        assert mla.read_device_error() == 0
+    finally:
+        del graph
