@@ -20,6 +20,12 @@
  *     caller's `workspace`.  Every call is asynchronous on `stream` (NULL = the legacy
  *     default stream), makes no host synchronisation and no allocation, and may
  *     therefore be captured in a CUDA graph.
+ *   - Stream order holds as for ordinary launches.  mla_decode_paged's kernel is a
+ *     programmatic dependent launch, and the metadata kernels let their dependent in at
+ *     their start.  Placed right after one of them, the attention kernel therefore sets
+ *     itself up while the metadata kernel still runs, and reads nothing before that
+ *     kernel has completed.  After any other kernel, copy or event it starts as an
+ *     ordinary launch would.
  *   - Arguments are validated on the host before any launch; a violation returns
  *     MLA_ERR_INVALID_ARG (or MLA_ERR_UNSUPPORTED for a valid but unimplemented
  *     combination) and launches nothing.  A CUDA launch error returns MLA_ERR_CUDA.
