@@ -15,10 +15,9 @@
 // Q = P - F blocks each, and the last piece takes the rest (1..Q blocks) -- a closed form
 // whose one division is needed only when a request spans more than two further parts.  One
 // thread runs that O(bs) recurrence, a short chain of compares per request; then one thread
-// per part reads its row off the per-request results by binary search: its first piece
-// belongs to the first request whose last part is >= i, its last to the last request
-// whose first part is <= i.  Batches larger than kPlannerSmemLens take the part-by-part
-// walk instead, reading the lengths from global memory.
+// per request writes the fields of the part rows that begin or end inside it.  Batches
+// larger than kPlannerSmemLens take the part-by-part walk instead, reading the lengths from
+// global memory.
 #pragma once
 #include "ptx.cuh"
 
@@ -150,44 +149,37 @@ __device__ __forceinline__ void plan_parts(LenFn len_of, int32_t bs, int32_t par
     }
     __syncthreads();
     if (threadIdx.x == 0) num_splits[0] = 0;
-    for (int b = threadIdx.x; b < bs; b += blockDim.x) num_splits[b + 1] = s_cum[b];
-    for (int i = threadIdx.x; i < parts; i += blockDim.x) {
-        int lo = 0, hi = bs;   // first request whose last part is >= i
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (s_lp[mid] >= i)
-                hi = mid;
-            else
-                lo = mid + 1;
+    // The part rows, scattered from the per-request results without a search.  Part i begins
+    // in the first request whose last part is >= i: request b for i in (lp[b-1], lp[b]].  It
+    // ends in the last request whose first part is <= i: request b for i in [fp[b], fp[b+1]),
+    // no further than lp[b].  Every part up to lp[bs-1] has one of each (no part in between is
+    // left empty: a request starts in the part the previous one ended in, or the next one);
+    // the parts after it are unused.
+    for (int b = threadIdx.x; b < bs; b += blockDim.x) {
+        num_splits[b + 1] = s_cum[b];
+        const int fpb = s_fp[b], lpb = s_lp[b], x0b = s_x0[b];
+        const int lp_prev = b > 0 ? s_lp[b - 1] : -1;
+        // (every index stays below parts, which the walk guarantees; the bounds only make sure)
+        const int last = min(lpb, parts - 1);
+        const int end_last = b + 1 < bs ? min(s_fp[b + 1] - 1, last) : last;
+        for (int i = lp_prev + 1; i <= last; ++i) {   // parts that begin in request b
+            int32_t* row = md + 8 * static_cast<int64_t>(i);
+            const int begin_s = i > fpb ? i - fpb : 0;
+            row[0] = b;
+            row[1] = begin_s > 0 ? x0b + (begin_s - 1) * Q : 0;
+            *reinterpret_cast<int4*>(row + 4) = make_int4(begin_s, 0, 0, 0);
         }
-        const int bb = lo;
-        int4 r0 = make_int4(bs, 0, bs, 0), r1 = make_int4(0, 0, 0, 0);
-        if (bb < bs) {
-            int begin_k = 0, begin_s = 0;
-            if (s_fp[bb] < i) {   // the part starts inside request bb
-                begin_s = i - s_fp[bb];
-                begin_k = s_x0[bb] + (begin_s - 1) * Q;
-            }
-            int lo2 = bb, hi2 = bs;   // last request whose first part is <= i
-            while (lo2 < hi2) {
-                const int mid = (lo2 + hi2) >> 1;
-                if (s_fp[mid] <= i)
-                    lo2 = mid + 1;
-                else
-                    hi2 = mid;
-            }
-            const int bl = lo2 - 1;
-            int end_b = bl + 1, end_k = 0;
-            if (s_lp[bl] > i) {   // the part ends inside request bl
-                end_b = bl;
-                end_k = s_x0[bl] + (i - s_fp[bl]) * Q;
-            }
-            r0 = make_int4(bb, begin_k, end_b, end_k);
-            r1 = make_int4(begin_s, 0, 0, 0);
+        for (int i = fpb; i <= end_last; ++i) {      // parts that end in request b
+            int32_t* row = md + 8 * static_cast<int64_t>(i);
+            const bool inside = lpb > i;
+            *reinterpret_cast<int2*>(row + 2) = make_int2(inside ? b : b + 1, inside ? x0b + (i - fpb) * Q : 0);
         }
+    }
+    const int used = bs > 0 ? min(s_lp[bs - 1] + 1, parts) : 0;
+    for (int i = used + threadIdx.x; i < parts; i += blockDim.x) {
         int4* row = reinterpret_cast<int4*>(md + 8 * static_cast<int64_t>(i));
-        row[0] = r0;
-        row[1] = r1;
+        row[0] = make_int4(bs, 0, bs, 0);
+        row[1] = make_int4(0, 0, 0, 0);
     }
 }
 

@@ -451,6 +451,29 @@ def test_planner_random_batches(mla):
         assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits differs (bs {bs}, parts {parts})"
 
 
+def test_planner_split_boundaries(mla):
+    """The walk's split count by comparisons (a piece past a part's budget spans one or two
+    further parts without a division, more with one): dense random batches whose requests are
+    about 0, 1, 2 or 3 budgets long, give or take a few blocks, with the part count set so the
+    budget lands near the one the lengths were drawn for.  Bit-exact against the oracle's
+    part-by-part walk."""
+    rng = np.random.default_rng(20261204)
+    for t in range(3000):
+        bs = int(rng.integers(1, 25))
+        b0 = int(rng.integers(3, 201))
+        nb = rng.integers(0, 4, size=bs) * b0 + rng.integers(-7, 8, size=bs)
+        nb = np.maximum(nb, 0)
+        lens = np.where(nb > 0, nb * 64 - rng.integers(0, 64, size=bs), 0)
+        total = int(nb.sum()) + 5 * bs
+        parts = int(min(148, max(1, round(total / b0) + int(rng.integers(-1, 2)))))
+        seqlens = torch.tensor(lens, dtype=torch.int32)
+        md, ns = mla.get_mla_metadata(seqlens.cuda(), 128, num_parts=parts)
+        ref_md, ref_ns = oracle.get_mla_metadata(seqlens.numpy(), parts)
+        assert np.array_equal(md.cpu().numpy(), ref_md), f"batch {t}: metadata differs (lens {lens.tolist()}, parts {parts})"
+        assert np.array_equal(ns.cpu().numpy(), ref_ns), f"batch {t}: num_splits differs (lens {lens.tolist()}, parts {parts})"
+    assert mla.read_device_error() == 0
+
+
 # ------------------------------------------------------------------ one-launch metadata
 @pytest.mark.parametrize("index", [1, 2, 3, 4, 5])
 def test_one_launch_metadata_matches_oracle(mla, index):
