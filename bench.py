@@ -64,7 +64,13 @@ def parse_args(argv=None):
                     help="time only the --config workload")
     ap.add_argument("--per-config-steps", type=int, default=50,
                     help="timed steps of each other workload in the per_config entries")
-    return ap.parse_args(argv)
+    ap.add_argument("--q-fp8", action="store_true",
+                    help="the fp8-cache workload (--config 4) with its queries handed over as e4m3 "
+                         "codes, the backend's fp8 recipe")
+    args = ap.parse_args(argv)
+    if args.q_fp8 and args.config != 4:
+        ap.error("--q-fp8 applies to the fp8-cache workload, --config 4")
+    return args
 
 
 def dist_env():
@@ -93,7 +99,8 @@ def job_value(world, kv_bytes_per_replica, step_ms):
     return world * kv_bytes_per_replica / (step_ms * 1e-3) / 1e9
 
 
-TRAFFIC_KEYS = {2: "deepseek_v3_decode", 3: "skewed_long_context", 4: "fp8_kv_decode", 5: "target_verify"}
+TRAFFIC_KEYS = {1: "tiny_decode", 2: "deepseek_v3_decode", 3: "skewed_long_context", 4: "fp8_kv_decode",
+                "4q8": "fp8_kv_fp8_q_decode", 5: "target_verify"}
 
 
 # The sources the decode kernel is built from: its body, the PTX helpers it inlines, and the
@@ -181,8 +188,9 @@ def algorithmic(wl):
 def workload_config(cfg_index, wl, world, flush_mb):
     from paged_kv_mla_create_b200.workloads import CONFIGS
     c = CONFIGS[cfg_index]
-    return {"workload": c["name"], "batch": wl.bs, "heads": wl.h, "q_len": wl.q_len,
-            "kv_dtype": "fp8_e4m3" if wl.is_fp8 else "bf16", "page": 64,
+    return {"workload": wl.name if wl.q_is_fp8 else c["name"], "batch": wl.bs, "heads": wl.h,
+            "q_len": wl.q_len, "kv_dtype": "fp8_e4m3" if wl.is_fp8 else "bf16",
+            "q_dtype": "fp8_e4m3" if wl.q_is_fp8 else "bf16", "page": 64,
             "head_dim": 576, "head_dim_v": 512,
             "l2": f"flushed between timed steps ({flush_mb} MB written, then another {flush_mb} MB read, "
                   "outside the step events: no input of the step and no dirty line left in L2)",
@@ -303,7 +311,7 @@ def run_reference(args):
         return 0
     import oracle
     from paged_kv_mla_create_b200 import workloads as W
-    wl = W.make_workload(args.config, seed=replica_seed(args.config, 0))
+    wl = W.make_workload(args.config, seed=replica_seed(args.config, 0), q_fp8=args.q_fp8)
     kv_bytes, _, _ = algorithmic(wl)
     total = wl.bs * wl.q_len * wl.h
     per_step = 120.0 / max(1, args.steps + args.warmup)
@@ -338,8 +346,8 @@ class Case:
         import paged_kv_mla_create_b200 as mla
         from paged_kv_mla_create_b200 import workloads as W
         self.mla, self.dev, self.cfg = mla, dev, cfg
-        # the committed DRAM capture that belongs to this workload's kernel (none for e4m3 q)
-        self.traffic_key = None if q_fp8 else cfg
+        # the committed DRAM capture that belongs to this workload's kernel
+        self.traffic_key = f"{cfg}q8" if q_fp8 else cfg
         self.host = host = W.make_workload(cfg, seed=seed, q_fp8=q_fp8)
         self.wl = host.to(dev)
         self.kv_bytes, self.q_bytes, self.flops = algorithmic(host)
@@ -589,8 +597,11 @@ class ExtendCase(Case):
 
 def config_entry(case, step_ms, attn_ms, meta_ms, clk, peaks, peak_src):
     attn_s = attn_ms * 1e-3
+    # metadata_us: the metadata call alone (its own graph, events around it); metadata_exposed_us:
+    # what it adds to a step replayed as one graph, where it overlaps the attention kernel's set-up
     return {"workload": case.host.name, "us_per_call": attn_ms * 1e3,
             "metadata_us": meta_ms * 1e3, "us_per_step": step_ms * 1e3,
+            "metadata_exposed_us": (step_ms - attn_ms) * 1e3,
             "kv_gbs_per_call": case.kv_bytes / attn_s / 1e9, "tflops": case.flops / attn_s / 1e12,
             "kv_bytes": case.kv_bytes, "q_bytes": case.q_bytes, "flops": case.flops,
             "roofline": roofline_entry(case.kv_bytes, case.q_bytes, case.flops, attn_s, peaks,
@@ -615,7 +626,7 @@ def run_b200(args):
     mla.library()
     peaks, peak_src = load_peaks()
 
-    case = Case(args.config, replica_seed(args.config, rank), dev, args.flush_mb)
+    case = Case(args.config, replica_seed(args.config, rank), dev, args.flush_mb, q_fp8=args.q_fp8)
     K = args.steps
     clocks = ClockSampler(gpu_id_for(dev))
     step_ms, attn_ms, meta_ms, clk = case.time_steps(K, args.warmup, world, clocks)
@@ -632,11 +643,11 @@ def run_b200(args):
     torch.cuda.empty_cache()
 
     # every other workload, with a short timed run each (its own clock record)
-    per_config = {str(args.config): head}
+    per_config = {f"{args.config}q8" if args.q_fp8 else str(args.config): head}
     if not args.no_per_config:
         # the five workloads, and the fp8-cache one with e4m3 queries (the backend's fp8 recipe)
         for cfg, q8 in ((1, False), (2, False), (3, False), (4, False), (4, True), (5, False)):
-            if cfg == args.config and not q8:
+            if cfg == args.config and q8 == args.q_fp8:
                 continue
             c = Case(cfg, replica_seed(cfg, rank), dev, args.flush_mb, q_fp8=q8)
             sm, am, mm, ck = c.time_steps(max(1, min(K, args.per_config_steps)), max(3, min(args.warmup, 5)),
@@ -668,10 +679,12 @@ def run_b200(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if host.is_fp8 else "bf16",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("e4m3/f16" if host.q_is_fp8 else "f16") if host.is_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(args.config, host, world, args.flush_mb),
         "us_per_call": head["us_per_call"], "metadata_us": head["metadata_us"],
+        "metadata_exposed_us": head["metadata_exposed_us"],
         "kv_gbs_per_call": head["kv_gbs_per_call"], "tflops": head["tflops"],
         "tensor_frac": head["tflops"] / peaks["bf16_tflops"],
         "roofline": head["roofline"],
