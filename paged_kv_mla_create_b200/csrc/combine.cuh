@@ -5,9 +5,9 @@
 //
 // Requests of 2 .. kFusedMergeMaxPieces pieces are merged inside the attention kernel, by the
 // piece that arrives last (merge_rows_cta_bulk, or folded into that piece's own epilogue); the
-// merge kernel takes requests of more pieces, a warp per query row: it reads the pieces' lse
-// values, then streams the pieces' 512 fp32 columns (16 per lane, as 4 float4; four pieces'
-// loads in flight at once, read once, evict-first) and writes bf16.
+// merge kernel takes requests of more pieces, a warp per 64-column slice of a query row: it reads
+// the pieces' lse values once, then streams the pieces' columns of its slice (2 per lane; 32
+// pieces' loads in flight at once, read once, evict-first) and writes bf16.
 #pragma once
 #include "ptx.cuh"
 
@@ -18,66 +18,70 @@ constexpr int kCombineWarps = 8;
 // CTA whose piece arrives last; the merge kernel serves requests of more pieces.
 constexpr int kFusedMergeMaxPieces = 4;
 
+// The merge kernel's unit of work: one 64-column slice of one query row, a warp, lane l holding
+// columns 64 slice + 2l, + 1.  A row's eight slices go to eight warps, so that a request of many
+// pieces (a long request split over every part) spreads over the whole grid: a warp per row left
+// its 128 rows to 16 of the 148 SMs, each warp streaming ~70 pieces x 2 KB in turn.
+constexpr int kMergeSliceCols = 64;
+constexpr int kMergeSlices = 512 / kMergeSliceCols;
+constexpr int kMergeRegPieces = 128;   // pieces whose lse values stay in registers (4 per lane)
+
 // Merge the n partial states (o_i, lse_i) of one query row (pieces s0 .. s0 + n - 1 of the
-// split slots) into bf16 o and its lse; one warp, lane l holding columns 4l + 128k + [0, 4).
-// The partials were written by an earlier grid, so the read-only path serves them.
-__device__ __forceinline__ void merge_row(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                                          int s0, int n, int rows, int row, __nv_bfloat16* __restrict__ out_row,
-                                          float* __restrict__ lse_out, int lane, uint64_t read_pol) {
+// split slots) into bf16 o, columns of `slice` only, and (slice 0) its lse.  Lane l reads the lse
+// of pieces l + 32k once; piece i's weight exp(lse_i - lse) is computed by lane i % 32 and
+// shuffled to the others.  The pieces go in rounds of 32 with all their loads in flight, and each
+// column sums w_i o_i in piece order.  The partials were written by an earlier grid, so the
+// read-only path serves them.
+__device__ __forceinline__ void merge_row_slice(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                                int s0, int n, int rows, int row, int slice,
+                                                __nv_bfloat16* __restrict__ out_row, float* __restrict__ lse_out,
+                                                int lane, uint64_t read_pol) {
     auto load_lse = [&](int i) -> float {
         const float* ptr = part_lse + (int64_t)(s0 + i) * rows + row;
         return *ptr;
     };
-    float m = -INFINITY;
-    for (int i = lane; i < n; i += 32) m = fmaxf(m, load_lse(i));
+    const int col = kMergeSliceCols * slice + 2 * lane;
+    float lr[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) lr[k] = lane + 32 * k < n ? load_lse(lane + 32 * k) : -INFINITY;
+    float m = fmaxf(fmaxf(lr[0], lr[1]), fmaxf(lr[2], lr[3]));
+    for (int i = lane + kMergeRegPieces; i < n; i += 32) m = fmaxf(m, load_lse(i));
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (m == -INFINITY) {
-        for (int c = lane; c < 64; c += 32) reinterpret_cast<uint4*>(out_row)[c] = make_uint4(0, 0, 0, 0);
-        if (lane == 0) *lse_out = -INFINITY;
+        reinterpret_cast<uint32_t*>(out_row)[col >> 1] = 0u;
+        if (slice == 0 && lane == 0) *lse_out = -INFINITY;
         return;
     }
     float sum = 0.f;
-    for (int i = lane; i < n; i += 32) sum += expf(load_lse(i) - m);
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float lse = m + logf(sum);
-    float acc[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    // pieces four at a time, all of their loads in flight before any is used
-    for (int i0 = 0; i0 < n; i0 += 4) {
-        float4 v[4][4];
-        float w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j;
-            w[j] = 0.f;
-            if (i < n) {
-                w[j] = expf(load_lse(i) - lse);
-                const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)(s0 + i) * rows + row) * 512);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    v[j][k] = ld_global_nc_v4_hint(src + lane + 32 * k, read_pol);
-            } else {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v[j][k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                acc[4 * k + 0] += w[j] * v[j][k].x;
-                acc[4 * k + 1] += w[j] * v[j][k].y;
-                acc[4 * k + 2] += w[j] * v[j][k].z;
-                acc[4 * k + 3] += w[j] * v[j][k].w;
-            }
-    }
-    uint2* dst = reinterpret_cast<uint2*>(out_row);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        dst[lane + 32 * k] = make_uint2(pack_bf16x2(acc[4 * k], acc[4 * k + 1]),
-                                        pack_bf16x2(acc[4 * k + 2], acc[4 * k + 3]));
-    if (lane == 0) *lse_out = lse;
+        if (lane + 32 * k < n) sum += expf(lr[k] - m);
+    for (int i = lane + kMergeRegPieces; i < n; i += 32) sum += expf(load_lse(i) - m);
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float lse = m + logf(sum);
+    float a0 = 0.f, a1 = 0.f;
+    // pieces c0 .. c0 + 31, lane l holding the weight of piece c0 + l
+    auto merge_round = [&](int c0, float wl) {
+        float2 v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            v[j] = c0 + j < n ? ld_global_nc_v2_hint(reinterpret_cast<const float2*>(
+                                    part_o + ((int64_t)(s0 + c0 + j) * rows + row) * 512 + col), read_pol)
+                              : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float w = __shfl_sync(0xffffffffu, wl, j);
+            a0 += w * v[j].x;
+            a1 += w * v[j].y;
+        }
+    };
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (32 * k < n) merge_round(32 * k, lane + 32 * k < n ? expf(lr[k] - lse) : 0.f);
+    for (int c0 = kMergeRegPieces; c0 < n; c0 += 32)
+        merge_round(c0, c0 + lane < n ? expf(load_lse(c0 + lane) - lse) : 0.f);
+    reinterpret_cast<uint32_t*>(out_row)[col >> 1] = pack_bf16x2(a0, a1);
+    if (slice == 0 && lane == 0) *lse_out = lse;
 }
 
 // Merge, with a whole CTA of kThreadsCta threads whose shared memory is idle, the n (2 ..
@@ -161,10 +165,10 @@ __device__ __forceinline__ bool merge_rows_cta_bulk(const float* __restrict__ pa
 // merged by the attention kernel, so the launch needs no host knowledge of the plan): each CTA
 // first stages num_splits in shared memory (one coalesced read, for up to kCombineStagedRequests
 // requests) and notes whether any request has that many pieces, then waits for the attention
-// grid; its warps then take (request, query row) pairs in turn, or the CTA returns at once when
-// nothing is left to merge.  num_splits comes from the metadata step: the attention kernel lets
-// this grid in only after its own wait for that step to complete, so num_splits is final and is
-// read while the attention kernel still runs.
+// grid; its warps then take (request, query row, column slice) units in turn, or the CTA returns
+// at once when nothing is left to merge.  num_splits comes from the metadata step: the attention
+// kernel lets this grid in only after its own wait for that step to complete, so num_splits is
+// final and is read while the attention kernel still runs.
 constexpr int kCombineStagedRequests = 4096;
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
@@ -190,15 +194,18 @@ combine_splits_kernel(const float* __restrict__ part_o, const float* __restrict_
     const uint64_t read_pol = l2_policy_evict_first();   // the partials are read once
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * kCombineWarps;
-    const int64_t total = (int64_t)bs * rows;
+    const int64_t per_req = (int64_t)rows * kMergeSlices;
+    const int64_t total = (int64_t)bs * per_req;
     for (int64_t idx = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5); idx < total; idx += warps) {
-        const int b = (int)(idx / rows);
-        const int row = (int)(idx - (int64_t)b * rows);
+        const int b = (int)(idx / per_req);
+        const int rs = (int)(idx - (int64_t)b * per_req);
+        const int row = rs / kMergeSlices, slice = rs - row * kMergeSlices;
         const int s0 = staged ? s_ns[b] : num_splits[b];
         const int n = (staged ? s_ns[b + 1] : num_splits[b + 1]) - s0;
         if (n <= kFusedMergeMaxPieces) continue;
         const int64_t out_row = (int64_t)b * rows + row;
-        merge_row(part_o, part_lse, s0, n, rows, row, out + out_row * 512, lse_out + out_row, lane, read_pol);
+        merge_row_slice(part_o, part_lse, s0, n, rows, row, slice, out + out_row * 512, lse_out + out_row, lane,
+                        read_pol);
     }
 }
 

@@ -434,8 +434,8 @@ mla_status_t mla_decode_paged(const void* q, int32_t q_dtype, int32_t bs, int32_
     // the attention kernel runs, it waits on the device for that grid to complete.
     cudaLaunchConfig_t cfg = {};
     {
-        const int64_t need = ((int64_t)bs * rows + mla::kCombineWarps - 1) / mla::kCombineWarps;
-        // as many CTAs as the attention grid (one per SM)
+        const int64_t need = ((int64_t)bs * rows * mla::kMergeSlices + mla::kCombineWarps - 1) / mla::kCombineWarps;
+        // a warp per (request, row, column slice), at most as many CTAs as the attention grid (one per SM)
         cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)grid.x * grid.y)));
     }
     cfg.blockDim = dim3(mla::kCombineWarps * 32);

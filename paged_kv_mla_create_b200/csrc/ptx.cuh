@@ -361,6 +361,13 @@ __device__ __forceinline__ float4 ld_global_nc_v4_hint(const float4* ptr, uint64
     return v;
 }
 
+// 8-byte read-only global load with an L2 cache policy.
+__device__ __forceinline__ float2 ld_global_nc_v2_hint(const float2* ptr, uint64_t pol) {
+    float2 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;" : "=f"(v.x), "=f"(v.y) : "l"(ptr), "l"(pol));
+    return v;
+}
+
 // Hint the L2 to fetch a tensor box ahead of its load (no shared memory involved).
 __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t c0, int32_t c1,
                                                 int32_t c2, int32_t c3) {
