@@ -124,6 +124,16 @@ def test_forced_splits(mla, parts):
     check_full(mla, W.make_case([2000, 33, 700, 4000, 129], h=128, seed=23, poison=True), parts)
 
 
+def test_more_parts_than_sms_and_a_request_of_many_pieces(mla):
+    """200 parts (400 CTAs, in waves: more than the SMs hold at once) split a 40000-token request
+    into 157 pieces. That is more than the merge kernel keeps in registers, so the lse values past
+    the first 128 pieces are reloaded and merged in further rounds."""
+    wl = W.make_case([40000, 3000], h=16, seed=31)
+    ref_md, ref_ns = oracle.get_mla_metadata(wl.cache_seqlens.numpy(), 200)
+    assert int(ref_ns[1] - ref_ns[0]) > 128
+    check_full(mla, wl, 200)
+
+
 @pytest.mark.parametrize("q_len,h", [(4, 128), (2, 128), (3, 16), (4, 40)])
 def test_target_verify(mla, q_len, h):
     check_full(mla, W.make_case([1000, 62, 129, 1], h=h, q_len=q_len, verify=True, seed=24,
