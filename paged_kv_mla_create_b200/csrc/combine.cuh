@@ -6,7 +6,7 @@
 // Requests of 2 .. kFusedMergeMaxPieces pieces are merged inside the attention kernel, by the
 // piece that arrives last (merge_rows_cta_bulk, or folded into that piece's own epilogue); the
 // merge kernel takes requests of more pieces, a warp per 64-column slice of a query row: it reads
-// the pieces' lse values once, then streams the pieces' columns of its slice (2 per lane; 64
+// the pieces' lse values once, then streams the pieces' columns of its slice (2 per lane; 32
 // pieces' loads in flight at once, read once, evict-first) and writes bf16.
 #pragma once
 #include "ptx.cuh"
@@ -29,9 +29,8 @@ constexpr int kMergeRegPieces = 128;   // pieces whose lse values stay in regist
 // Merge the n partial states (o_i, lse_i) of one query row (pieces s0 .. s0 + n - 1 of the
 // split slots) into bf16 o, columns of `slice` only, and (slice 0) its lse.  Lane l reads the lse
 // of pieces l + 32k once; piece i's weight exp(lse_i - lse) is computed by lane i % 32 and
-// shuffled to the others.  The pieces go in rounds of 64 with all their loads in flight (two
-// rounds for a request split over every part of the grid; rounds of 32 took ~2 us longer on the
-// skewed workload), and each column sums w_i o_i in piece order.  The partials were written by an earlier grid, so the
+// shuffled to the others.  The pieces go in rounds of 32 with all their loads in flight, and each
+// column sums w_i o_i in piece order.  The partials were written by an earlier grid, so the
 // read-only path serves them.
 __device__ __forceinline__ void merge_row_slice(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                                 int s0, int n, int rows, int row, int slice,
@@ -61,27 +60,26 @@ __device__ __forceinline__ void merge_row_slice(const float* __restrict__ part_o
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     const float lse = m + logf(sum);
     float a0 = 0.f, a1 = 0.f;
-    // pieces c0 .. c0 + 63, lane l holding the weights of pieces c0 + l and c0 + 32 + l
-    auto merge_round = [&](int c0, float wl0, float wl1) {
-        float2 v[64];
+    // pieces c0 .. c0 + 31, lane l holding the weight of piece c0 + l
+    auto merge_round = [&](int c0, float wl) {
+        float2 v[32];
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
+        for (int j = 0; j < 32; ++j)
             v[j] = c0 + j < n ? ld_global_nc_v2_hint(reinterpret_cast<const float2*>(
                                     part_o + ((int64_t)(s0 + c0 + j) * rows + row) * 512 + col), read_pol)
                               : make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            const float w = __shfl_sync(0xffffffffu, j < 32 ? wl0 : wl1, j & 31);
+        for (int j = 0; j < 32; ++j) {
+            const float w = __shfl_sync(0xffffffffu, wl, j);
             a0 += w * v[j].x;
             a1 += w * v[j].y;
         }
     };
-    auto wreg = [&](int k) { return lane + 32 * k < n ? expf(lr[k] - lse) : 0.f; };
-    if (n > 0) merge_round(0, wreg(0), wreg(1));
-    if (n > 64) merge_round(64, wreg(2), wreg(3));
-    for (int c0 = kMergeRegPieces; c0 < n; c0 += 64)
-        merge_round(c0, c0 + lane < n ? expf(load_lse(c0 + lane) - lse) : 0.f,
-                    c0 + 32 + lane < n ? expf(load_lse(c0 + 32 + lane) - lse) : 0.f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (32 * k < n) merge_round(32 * k, lane + 32 * k < n ? expf(lr[k] - lse) : 0.f);
+    for (int c0 = kMergeRegPieces; c0 < n; c0 += 32)
+        merge_round(c0, c0 + lane < n ? expf(load_lse(c0 + lane) - lse) : 0.f);
     reinterpret_cast<uint32_t*>(out_row)[col >> 1] = pack_bf16x2(a0, a1);
     if (slice == 0 && lane == 0) *lse_out = lse;
 }
