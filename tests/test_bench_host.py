@@ -47,3 +47,29 @@ def test_roofline_fp8_cache_can_be_hbm_bound():
 def test_roofline_fallback_peak_is_named():
     r = bench.roofline_entry(1e9, 0.0, 1e9, 1e-3, bench.FALLBACK_PEAKS, "fallback", False, None)
     assert r["peak_source"] == "fallback"
+
+
+def test_q_fp8_only_with_the_fp8_cache_workload():
+    import pytest
+    assert bench.parse_args(["--config", "4", "--q-fp8"]).q_fp8
+    assert not bench.parse_args([]).q_fp8
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--config", "2", "--q-fp8"])
+
+
+def test_config_entry_reports_what_metadata_adds_to_the_step():
+    class _Host:
+        name = "w"
+        is_fp8 = False
+
+    class _Case:
+        host = _Host()
+        kv_bytes, q_bytes, flops = 183e6, 9.4e6, 44e9
+        traffic_key = None
+
+    e = bench.config_entry(_Case(), 0.0797, 0.0739, 0.0103, None, PEAKS, "measured")
+    assert math.isclose(e["us_per_step"], 79.7)
+    assert math.isclose(e["us_per_call"], 73.9)
+    assert math.isclose(e["metadata_us"], 10.3)
+    assert math.isclose(e["metadata_exposed_us"], 79.7 - 73.9)
+    json.dumps(e)
